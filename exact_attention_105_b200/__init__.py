@@ -1,0 +1,156 @@
+"""Python binding of the sm_100a exact-attention library (libattn_sm100.so).
+
+The binding only marshals arguments. It takes shapes, data pointers and the
+current CUDA stream from torch tensors and calls the C ABI declared in
+``include/attn.h``. All arithmetic runs in the library's CUDA kernels. There
+is no fallback: if the shared library is missing or the device is not an
+sm_100 part, every call raises.
+
+Layout: q, o, dO, dq are [B, Hq, N, d]. k, v, dk, dv are [B, Hkv, N, d].
+All are contiguous bfloat16 CUDA tensors. lse is [B, Hq, N] float32.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libattn_sm100.so")
+
+ATTN_OK, ATTN_ERR_ARG, ATTN_ERR_UNSUPPORTED, ATTN_ERR_CUDA, ATTN_ERR_TIMEOUT = range(5)
+_STATUS_NAMES = {0: "ATTN_OK", 1: "ATTN_ERR_ARG", 2: "ATTN_ERR_UNSUPPORTED",
+                 3: "ATTN_ERR_CUDA", 4: "ATTN_ERR_TIMEOUT"}
+
+# Every symbol include/attn.h declares, with its ctypes signature.
+_P, _I, _F, _SZ = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+SIGNATURES = {
+    "attn_fwd": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _I, _P]),
+    "attn_bwd": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _SZ,
+                      _I, _I, _I, _I, _I, _F, _I, _P]),
+    "attn_bwd_workspace_size": (_SZ, [_I, _I, _I, _I]),
+    "attn_check_status": (_I, [_P]),
+    "attn_get_last_error": (ctypes.c_char_p, []),
+    "attn_abi_version": (_I, []),
+}
+
+_lib = None
+
+
+class AttnError(RuntimeError):
+    """A non-OK status from the library, with its message."""
+
+    def __init__(self, status: int, message: str):
+        super().__init__(f"{_STATUS_NAMES.get(status, status)}: {message}")
+        self.status = status
+
+
+def load_library():
+    """Load (once) and return the ctypes handle; raise if it was never built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(
+                f"{LIB_PATH} is missing: build it with `python -m exact_attention_105_b200.build` "
+                "(there is no CPU fallback)")
+        lib = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in SIGNATURES.items():
+            fn = getattr(lib, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = lib
+    return _lib
+
+
+def _check(status: int):
+    if status != ATTN_OK:
+        msg = load_library().attn_get_last_error().decode(errors="replace")
+        raise AttnError(status, msg)
+
+
+def _stream_handle(stream):
+    import torch
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _dev_ptr(t, name):
+    import torch
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor (the library takes device pointers)")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _check_dtype(t, dtype, name):
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+
+
+def attn_fwd(q, k, v, o=None, lse=None, scale=None, causal=False, stream=None):
+    """Forward pass; returns (o, lse). Allocates o/lse with torch if not given."""
+    import torch
+    B, Hq, N, d = q.shape
+    Hkv = k.shape[1]
+    if k.shape != (B, Hkv, N, d) or v.shape != k.shape:
+        raise ValueError(f"k/v shape {tuple(k.shape)}/{tuple(v.shape)} does not match q {tuple(q.shape)}")
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _check_dtype(t, torch.bfloat16, n)
+    if o is None:
+        o = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, Hq, N), dtype=torch.float32, device=q.device)
+    _check_dtype(o, torch.bfloat16, "o")
+    _check_dtype(lse, torch.float32, "lse")
+    if o.shape != q.shape or lse.shape != (B, Hq, N):
+        raise ValueError("o/lse shape mismatch")
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    lib = load_library()
+    _check(lib.attn_fwd(_dev_ptr(q, "q"), _dev_ptr(k, "k"), _dev_ptr(v, "v"), _dev_ptr(o, "o"),
+                        _dev_ptr(lse, "lse"), B, Hq, Hkv, N, d, scale, int(bool(causal)),
+                        _stream_handle(stream)))
+    return o, lse
+
+
+def attn_bwd_workspace_size(B, Hq, N, d) -> int:
+    return int(load_library().attn_bwd_workspace_size(B, Hq, N, d))
+
+
+def attn_bwd(q, k, v, o, lse, dO, dq=None, dk=None, dv=None, workspace=None, scale=None,
+             causal=False, stream=None):
+    """Backward pass; returns (dq, dk, dv). Allocates outputs/workspace if not given."""
+    import torch
+    B, Hq, N, d = q.shape
+    Hkv = k.shape[1]
+    if k.shape != (B, Hkv, N, d) or v.shape != k.shape or o.shape != q.shape \
+            or dO.shape != q.shape or lse.shape != (B, Hq, N):
+        raise ValueError("shape mismatch among q, k, v, o, lse, dO")
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (o, "o"), (dO, "dO")):
+        _check_dtype(t, torch.bfloat16, n)
+    _check_dtype(lse, torch.float32, "lse")
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    for t, n, ref in ((dq, "dq", q), (dk, "dk", k), (dv, "dv", v)):
+        _check_dtype(t, torch.bfloat16, n)
+        if t.shape != ref.shape:
+            raise ValueError(f"{n} shape mismatch")
+    need = attn_bwd_workspace_size(B, Hq, N, d)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    lib = load_library()
+    _check(lib.attn_bwd(_dev_ptr(q, "q"), _dev_ptr(k, "k"), _dev_ptr(v, "v"), _dev_ptr(o, "o"),
+                        _dev_ptr(lse, "lse"), _dev_ptr(dO, "dO"), _dev_ptr(dq, "dq"),
+                        _dev_ptr(dk, "dk"), _dev_ptr(dv, "dv"), _dev_ptr(workspace, "workspace"),
+                        workspace.numel() * workspace.element_size(),
+                        B, Hq, Hkv, N, d, scale, int(bool(causal)), _stream_handle(stream)))
+    return dq, dk, dv
+
+
+def attn_check_status(stream=None):
+    """Synchronise the stream and raise AttnError if a kernel reported a timeout."""
+    _check(load_library().attn_check_status(_stream_handle(stream)))

@@ -1,0 +1,265 @@
+// C-ABI entry points of the attention library (declared in include/attn.h).
+//
+// This file is the only translation unit: it includes every kernel, so the
+// device status word has exactly one definition. Host work per call is
+// argument validation, tensor-map encoding (three to five 3-D maps) and the
+// kernel launches; nothing is allocated and nothing is synchronised except in
+// attn_check_status().
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/attn.h"
+#include "attn_bwd.cuh"
+#include "attn_fwd.cuh"
+#include "sm100.cuh"
+
+namespace {
+
+thread_local char g_last_error[512] = "";
+
+attn_status fail(attn_status code, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_last_error, sizeof(g_last_error), fmt, ap);
+  va_end(ap);
+  return code;
+}
+
+attn_status cuda_fail(cudaError_t e, const char* what) {
+  return fail(ATTN_ERR_CUDA, "%s: %s (%s)", what, cudaGetErrorName(e), cudaGetErrorString(e));
+}
+
+// ---------------------------------------------------------------- driver entry
+// cuTensorMapEncodeTiled is a driver API call; it is fetched through the
+// runtime so the library links only the static CUDA runtime and can be
+// loaded (for symbol checks) on a machine without a GPU driver.
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn g_encode = nullptr;
+attn_status g_init_status = ATTN_OK;
+char g_init_msg[256] = "";
+std::once_flag g_init_once;
+
+void init_once() {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) {
+    g_init_status = ATTN_ERR_CUDA;
+    snprintf(g_init_msg, sizeof(g_init_msg), "no CUDA device: %s", cudaGetErrorString(e));
+    return;
+  }
+  cudaDeviceProp prop;
+  e = cudaGetDeviceProperties(&prop, dev);
+  if (e != cudaSuccess || prop.major != 10 || prop.minor != 0) {
+    g_init_status = ATTN_ERR_CUDA;
+    snprintf(g_init_msg, sizeof(g_init_msg),
+             "this library is built for sm_100a (B200); device %d is sm_%d%d", dev, prop.major,
+             prop.minor);
+    return;
+  }
+  cudaDriverEntryPointQueryResult q;
+  void* fn = nullptr;
+  e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q);
+  if (e != cudaSuccess || q != cudaDriverEntryPointSuccess || fn == nullptr) {
+    g_init_status = ATTN_ERR_CUDA;
+    snprintf(g_init_msg, sizeof(g_init_msg), "cuTensorMapEncodeTiled unavailable");
+    return;
+  }
+  g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+}
+
+attn_status ensure_init() {
+  std::call_once(g_init_once, init_once);
+  if (g_init_status != ATTN_OK) return fail(g_init_status, "%s", g_init_msg);
+  return ATTN_OK;
+}
+
+// 3-D tensor map over a contiguous [BH, N, d] bf16 tensor with a box of
+// 64 x 128 x 1 (one 128-row, 128-byte-wide column block) and 128-byte
+// swizzle. Rows past N of a head read as zeros, never as the next head.
+attn_status make_map(CUtensorMap* map, const void* base, int d, int N, int BH) {
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N),
+                        static_cast<cuuint64_t>(BH)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2,
+                           static_cast<cuuint64_t>(d) * 2 * static_cast<cuuint64_t>(N)};
+  cuuint32_t box[3] = {64, 128, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims,
+                        strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(ATTN_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+  return ATTN_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Null, alignment and memory-kind checks for the tensor arguments. A host
+// pointer handed to a kernel would fault the GPU, so it is rejected here.
+attn_status check_ptrs(const void* const* ptrs, const char* const* names, int n) {
+  for (int i = 0; i < n; ++i) {
+    if (ptrs[i] == nullptr) return fail(ATTN_ERR_ARG, "%s is null", names[i]);
+    if (!aligned16(ptrs[i])) return fail(ATTN_ERR_ARG, "%s is not 16-byte aligned", names[i]);
+  }
+  for (int i = 0; i < n; ++i) {
+    cudaPointerAttributes pa;
+    cudaError_t e = cudaPointerGetAttributes(&pa, ptrs[i]);
+    if (e != cudaSuccess) {
+      cudaGetLastError();
+      return fail(ATTN_ERR_ARG, "%s is not a CUDA pointer (%s)", names[i], cudaGetErrorName(e));
+    }
+    if (pa.type != cudaMemoryTypeDevice && pa.type != cudaMemoryTypeManaged)
+      return fail(ATTN_ERR_ARG, "%s is not device memory", names[i]);
+  }
+  return ATTN_OK;
+}
+
+// Shape checks shared by forward and backward. Returns ATTN_OK and sets
+// *empty when there is nothing to compute.
+attn_status check_shape(int B, int Hq, int Hkv, int N, int d, float scale, bool* empty) {
+  *empty = false;
+  if (B < 0 || N < 0) return fail(ATTN_ERR_ARG, "B and N must be >= 0 (got B=%d N=%d)", B, N);
+  if (Hq < 1 || Hkv < 1) return fail(ATTN_ERR_ARG, "Hq and Hkv must be >= 1 (got %d, %d)", Hq, Hkv);
+  if (Hq % Hkv != 0)
+    return fail(ATTN_ERR_ARG, "Hq (%d) must be divisible by Hkv (%d) for MQA/GQA", Hq, Hkv);
+  if (d != 64 && d != 128)
+    return fail(ATTN_ERR_UNSUPPORTED, "head dim %d not supported (built: 64, 128)", d);
+  if (!(scale > 0.f) || !std::isfinite(scale))
+    return fail(ATTN_ERR_ARG, "scale must be finite and > 0 (got %g)", (double)scale);
+  if (static_cast<long long>(B) * Hq > 0x7FFFFFFFLL)
+    return fail(ATTN_ERR_ARG, "B*Hq too large");
+  if (N > (1 << 24)) return fail(ATTN_ERR_ARG, "N=%d exceeds the supported maximum 2^24", N);
+  if (B == 0 || N == 0) *empty = true;
+  return ATTN_OK;
+}
+
+template <int D, bool CAUSAL>
+attn_status launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                       void* o, float* lse, int B, int Hq, int Hkv, int N, float scale,
+                       cudaStream_t stream) {
+  using Cfg = attn::FwdCfg<D>;
+  auto kern = attn::fwd_kernel<D, CAUSAL>;
+  static std::once_flag attr_once;
+  static cudaError_t attr_err = cudaSuccess;
+  static int launch_regs = 0;
+  std::call_once(attr_once, [&] {
+    attr_err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    Cfg::kSmemAlloc);
+    cudaFuncAttributes fa;
+    if (attr_err == cudaSuccess) attr_err = cudaFuncGetAttributes(&fa, kern);
+    if (attr_err == cudaSuccess) launch_regs = fa.numRegs;
+  });
+  if (attr_err != cudaSuccess) return cuda_fail(attr_err, "cudaFuncSetAttribute(fwd)");
+  // The kernel rebalances registers between warpgroups with setmaxnreg; that
+  // split is only valid for the launch register count it was written for.
+  if (launch_regs != attn::kFwdRegsLaunch)
+    return fail(ATTN_ERR_CUDA, "fwd kernel built with %d registers/thread, expected %d",
+                launch_regs, attn::kFwdRegsLaunch);
+  dim3 grid(B * Hq, (N + 255) / 256);
+  const float scale_log2 = scale * 1.4426950408889634f;
+  kern<<<grid, Cfg::kThreads, Cfg::kSmemAlloc, stream>>>(
+      mq, mk, mv, static_cast<__nv_bfloat16*>(o), lse, Hq, Hq / Hkv, N, scale_log2);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "fwd kernel launch");
+  return ATTN_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int attn_abi_version(void) { return 100; }
+
+const char* attn_get_last_error(void) { return g_last_error; }
+
+attn_status attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                     int Hq, int Hkv, int N, int d, float scale, int causal,
+                     attn_stream_t stream_) {
+  g_last_error[0] = '\0';
+  bool empty = false;
+  attn_status st = check_shape(B, Hq, Hkv, N, d, scale, &empty);
+  if (st != ATTN_OK) return st;
+  if (causal != 0 && causal != 1) return fail(ATTN_ERR_ARG, "causal must be 0 or 1");
+  if (empty) return ATTN_OK;
+  const void* ptrs[5] = {q, k, v, o, lse};
+  const char* names[5] = {"q", "k", "v", "o", "lse"};
+  for (int i = 0; i < 5; ++i) {
+    if (ptrs[i] == nullptr) return fail(ATTN_ERR_ARG, "%s is null", names[i]);
+    if (!aligned16(ptrs[i])) return fail(ATTN_ERR_ARG, "%s is not 16-byte aligned", names[i]);
+  }
+  st = ensure_init();
+  if (st != ATTN_OK) return st;
+  if ((st = check_ptrs(ptrs, names, 5)) != ATTN_OK) return st;
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+  CUtensorMap mq, mk, mv;
+  if ((st = make_map(&mq, q, d, N, B * Hq)) != ATTN_OK) return st;
+  if ((st = make_map(&mk, k, d, N, B * Hkv)) != ATTN_OK) return st;
+  if ((st = make_map(&mv, v, d, N, B * Hkv)) != ATTN_OK) return st;
+  if (d == 64)
+    return causal ? launch_fwd<64, true>(mq, mk, mv, o, lse, B, Hq, Hkv, N, scale, stream)
+                  : launch_fwd<64, false>(mq, mk, mv, o, lse, B, Hq, Hkv, N, scale, stream);
+  return causal ? launch_fwd<128, true>(mq, mk, mv, o, lse, B, Hq, Hkv, N, scale, stream)
+                : launch_fwd<128, false>(mq, mk, mv, o, lse, B, Hq, Hkv, N, scale, stream);
+}
+
+size_t attn_bwd_workspace_size(int B, int Hq, int N, int d) {
+  (void)d;
+  if (B <= 0 || Hq <= 0 || N <= 0) return 0;
+  return static_cast<size_t>(B) * Hq * N * sizeof(float);
+}
+
+attn_status attn_bwd(const void* q, const void* k, const void* v, const void* o,
+                     const float* lse, const void* dO, void* dq, void* dk, void* dv,
+                     void* workspace, size_t workspace_bytes, int B, int Hq, int Hkv, int N,
+                     int d, float scale, int causal, attn_stream_t stream_) {
+  g_last_error[0] = '\0';
+  bool empty = false;
+  attn_status st = check_shape(B, Hq, Hkv, N, d, scale, &empty);
+  if (st != ATTN_OK) return st;
+  if (causal != 0 && causal != 1) return fail(ATTN_ERR_ARG, "causal must be 0 or 1");
+  if (empty) return ATTN_OK;
+  const void* ptrs[10] = {q, k, v, o, lse, dO, dq, dk, dv, workspace};
+  const char* names[10] = {"q", "k", "v", "o", "lse", "dO", "dq", "dk", "dv", "workspace"};
+  for (int i = 0; i < 10; ++i) {
+    if (ptrs[i] == nullptr) return fail(ATTN_ERR_ARG, "%s is null", names[i]);
+    if (!aligned16(ptrs[i])) return fail(ATTN_ERR_ARG, "%s is not 16-byte aligned", names[i]);
+  }
+  const size_t need = attn_bwd_workspace_size(B, Hq, N, d);
+  if (workspace_bytes < need)
+    return fail(ATTN_ERR_ARG, "workspace is %zu bytes, needs %zu", workspace_bytes, need);
+  st = ensure_init();
+  if (st != ATTN_OK) return st;
+  if ((st = check_ptrs(ptrs, names, 10)) != ATTN_OK) return st;
+  (void)stream_;
+  return fail(ATTN_ERR_UNSUPPORTED, "attn_bwd: not built yet");
+}
+
+attn_status attn_check_status(attn_stream_t stream_) {
+  g_last_error[0] = '\0';
+  attn_status st = ensure_init();
+  if (st != ATTN_OK) return st;
+  cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream_));
+  if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+  int word = 0;
+  e = cudaMemcpyFromSymbol(&word, attn::g_attn_device_status, sizeof(int));
+  if (e != cudaSuccess) return cuda_fail(e, "read status word");
+  if (word != 0) {
+    const int zero = 0;
+    e = cudaMemcpyToSymbol(attn::g_attn_device_status, &zero, sizeof(int));
+    if (e != cudaSuccess) return cuda_fail(e, "clear status word");
+    return fail(ATTN_ERR_TIMEOUT, "kernel gave up on a pipeline wait (code %d, site %d)",
+                word & 0xFF, (word >> 8) & 0xFF);
+  }
+  return ATTN_OK;
+}
+
+}  // extern "C"

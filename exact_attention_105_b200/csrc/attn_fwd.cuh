@@ -1,0 +1,400 @@
+// Forward kernel: O = softmax(Q K^T * scale [causal]) V and lse, one CTA per
+// (batch*head, 256-row query block), on tcgen05 tensor cores.
+//
+// Method: hysenlabs.com "FlashAttention: exakte Attention-Kernel fuer CUDA
+// und ROCm", section "Die Schnittstellen von flash_attn_func bis KV-Cache",
+// gives the formula. unite.ai "Was ist FlashAttention?", five-stage map:
+//   stage 1: Q, K and V are cut into 128-row tiles;
+//   stage 2: TMA brings each tile into shared memory (a ring of slots);
+//   stage 3: S = Q K^T is computed per tile into tensor memory, then a
+//            running row max / row sum normalises it (online softmax);
+//   stage 4: O += P V accumulates in tensor memory, so the N x N matrix is
+//            never materialised;
+//   stage 5: the grid is scheduled for the B200, heavy causal blocks first.
+//
+// CTA layout (384 threads, 12 warps):
+//   warps 0-3  softmax warpgroup for query tile 0 (rows 0..127 of the block)
+//   warps 4-7  softmax warpgroup for query tile 1 (rows 128..255)
+//   warp 8     TMA producer (one elected lane)
+//   warp 9     TMEM allocator and MMA issuer (one elected lane)
+//   warps 10-11 idle
+// Thread r of a softmax warpgroup owns TMEM lane r, i.e. query row r of its
+// tile. That is the 32x32b access pattern: warp w%4 reads lanes 32*(w%4)...
+//
+// Tensor memory (512 columns x 128 lanes x 32 bit):
+//   [  0,128) S0 fp32; P0 (bf16 pairs) overwrites S0 columns [64,128)
+//   [128,256) S1 fp32; P1 overwrites S1 columns [64,128)
+//   [256,256+D) O0 fp32 accumulator, [384,384+D) O1 fp32 accumulator
+// P_t(j) is read by the PV MMA, and the next S_t(j+1) MMA overwrites the
+// same columns. Both MMAs come from the same issuing thread, in that order,
+// and the tensor pipe executes one thread's MMAs in issue order.
+//
+// Shared memory: Q0, Q1 tiles, then a ring of NSTAGE K/V slots. K_j and V_j
+// take turns: K0, V0, K1, V1, ... Each 128 x D tile is stored as D/64
+// column blocks of 128 rows x 128 bytes, 128-byte swizzled, exactly as the
+// TMA writes it. That is the canonical K-major SW128 layout for Q and K and
+// the MN-major SW128 layout for V.
+#pragma once
+
+#include "sm100.cuh"
+
+namespace attn {
+
+template <int D>
+struct FwdCfg {
+  static_assert(D == 64 || D == 128, "head dim");
+  static constexpr int kTileBytes = 128 * D * 2;          // one 128 x D bf16 tile
+  static constexpr int kStages = (D == 128) ? 4 : 6;      // K/V ring slots
+  static constexpr int kQOff = 0;
+  static constexpr int kKVOff = 2 * kTileBytes;
+  static constexpr int kBarOff = kKVOff + kStages * kTileBytes;
+  // q_full[2] kv_full[S] kv_empty[S] s_full[2] p_full[2] o_full[2] mma_done[1]
+  static constexpr int kNumBars = 2 + 2 * kStages + 2 + 2 + 2 + 1;
+  static constexpr int kMiscOff = kBarOff + kNumBars * 8;
+  static constexpr int kBytes = kMiscOff + 16;
+  static constexpr int kSmemAlloc = kBytes + 1024;         // slack for 1024-B alignment
+  static constexpr int kThreads = 384;
+  static constexpr uint32_t kTxBytes = kTileBytes;
+};
+
+// Wait-site ids reported in the status word when a wait times out.
+enum FwdSite : int {
+  kSiteQFull = 1, kSiteKVFull = 2, kSiteKVEmpty = 3, kSiteSFull = 4, kSitePFull = 5,
+  kSiteOFull = 6, kSiteDrain = 7
+};
+
+// Bounded wait that ignores the abort flag: used only to let this thread's
+// own in-flight asynchronous copies / MMAs land before the CTA exits.
+__device__ __forceinline__ void mbar_wait_drain(uint64_t* bar, uint32_t parity) {
+  const unsigned long long t0 = global_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (global_ns() - t0 > kWaitTimeoutNs) {
+      atomicCAS(&g_attn_device_status, 0, kDevTimeout | (kSiteDrain << 8));
+      return;
+    }
+  }
+}
+
+__device__ __forceinline__ float u2f(uint32_t x) { return __uint_as_float(x); }
+__device__ __forceinline__ uint32_t f2u(float x) { return __float_as_uint(x); }
+
+// Register split: launched at kFwdRegsLaunch per thread (384 threads fill the
+// 64K register file); warpgroup 2 (producer, MMA, idle) drops to
+// kFwdRegsSmall and the two softmax warpgroups grow to kFwdRegsSoftmax.
+// 2 * 216 + 72 = 3 * 168. The host refuses to launch if ptxas allocated a
+// different launch count, since the grow would otherwise never be granted.
+constexpr int kFwdRegsLaunch = 168;
+constexpr int kFwdRegsSoftmax = 216;
+constexpr int kFwdRegsSmall = 72;
+static_assert(2 * kFwdRegsSoftmax + kFwdRegsSmall <= 3 * kFwdRegsLaunch, "register split");
+
+template <int D, bool CAUSAL>
+__global__ void __launch_bounds__(384, 1)
+fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+           const __grid_constant__ CUtensorMap tm_v, __nv_bfloat16* __restrict__ out,
+           float* __restrict__ lse_out, int Hq, int group, int N, float scale_log2) {
+  using C = FwdCfg<D>;
+  constexpr int NS = C::kStages;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  const uint32_t sbase = smem_u32(smem);
+
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kBarOff);
+  uint64_t* q_full = bars;
+  uint64_t* kv_full = q_full + 2;
+  uint64_t* kv_empty = kv_full + NS;
+  uint64_t* s_full = kv_empty + NS;
+  uint64_t* p_full = s_full + 2;
+  uint64_t* o_full = p_full + 2;
+  uint64_t* mma_done = o_full + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kMiscOff);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kMiscOff + 4);
+
+  const int warp = warp_id();
+  const int lane = lane_id();
+  const int bh = blockIdx.x;                       // b * Hq + hq
+  const int b = bh / Hq;
+  const int hq = bh - b * Hq;
+  const int bh_kv = b * (Hq / group) + hq / group; // GQA: contiguous head groups
+  const int mb = gridDim.y - 1 - blockIdx.y;       // heaviest causal blocks launch first
+  const int nkv = (N + 127) >> 7;
+
+  int n_t[2];
+#pragma unroll
+  for (int t = 0; t < 2; ++t) {
+    const int r0 = mb * 256 + t * 128;
+    n_t[t] = (r0 >= N) ? 0 : (CAUSAL ? min(nkv, (r0 >> 7) + 1) : nkv);
+  }
+  const int n_max = max(n_t[0], n_t[1]);
+
+  if (threadIdx.x == 0) {
+    mbar_init(&q_full[0], 1);
+    mbar_init(&q_full[1], 1);
+    for (int i = 0; i < NS; ++i) {
+      mbar_init(&kv_full[i], 1);
+      mbar_init(&kv_empty[i], 1);
+    }
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(&s_full[t], 1);
+      mbar_init(&p_full[t], 128);
+      mbar_init(&o_full[t], 1);
+    }
+    mbar_init(mma_done, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 9) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp >= 8) {
+    regs_shrink<kFwdRegsSmall>();
+    if (warp == 8 && lane == 0) {
+      // ---------------------------------------------------------- producer
+      tma_prefetch_desc(&tm_q);
+      tma_prefetch_desc(&tm_k);
+      tma_prefetch_desc(&tm_v);
+#pragma unroll
+      for (int t = 0; t < 2; ++t) {
+        if (n_t[t] > 0) {
+          mbar_expect_tx(&q_full[t], C::kTxBytes);
+#pragma unroll
+          for (int a = 0; a < D / 64; ++a)
+            tma_load_3d(smem + C::kQOff + t * C::kTileBytes + a * 16384, &tm_q, &q_full[t],
+                        a * 64, mb * 256 + t * 128, bh);
+        }
+      }
+      uint32_t issued = 0;
+      bool ok = true;
+      for (int j = 0; j < n_max && ok; ++j) {
+        for (int w = 0; w < 2; ++w) {
+          const uint32_t s = issued % NS;
+          const uint32_t round = issued / NS;
+          if (round > 0 && !mbar_wait(&kv_empty[s], (round - 1) & 1u, abort_flag, kSiteKVEmpty)) {
+            ok = false;
+            break;
+          }
+          mbar_expect_tx(&kv_full[s], C::kTxBytes);
+#pragma unroll
+          for (int a = 0; a < D / 64; ++a)
+            tma_load_3d(smem + C::kKVOff + s * C::kTileBytes + a * 16384, w ? &tm_v : &tm_k,
+                        &kv_full[s], a * 64, j * 128, bh_kv);
+          ++issued;
+        }
+      }
+      // Let every copy this thread started land before the CTA can exit.
+#pragma unroll
+      for (int t = 0; t < 2; ++t)
+        if (n_t[t] > 0) mbar_wait_drain(&q_full[t], 0);
+      const uint32_t first = issued > (uint32_t)NS ? issued - NS : 0u;
+      for (uint32_t i = first; i < issued; ++i) mbar_wait_drain(&kv_full[i % NS], (i / NS) & 1u);
+    } else if (warp == 9 && lane == 0) {
+      // ---------------------------------------------------------- MMA issuer
+      constexpr uint32_t kIdescQK = idesc_bf16_f32(128, 128, 0, 0);
+      constexpr uint32_t kIdescPV = idesc_bf16_f32(128, D, 0, 1);
+      auto issue_qk = [&](int t, uint32_t slot) {
+        const uint32_t qa = sbase + C::kQOff + t * C::kTileBytes;
+        const uint32_t ka = sbase + C::kKVOff + slot * C::kTileBytes;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+          mma_ss(tmem + t * 128, sdesc_sw128(qa + off, 16, 1024), sdesc_sw128(ka + off, 16, 1024),
+                 kIdescQK, kk > 0 ? 1u : 0u);
+        }
+      };
+      auto issue_pv = [&](int t, uint32_t slot, bool acc) {
+        const uint32_t va = sbase + C::kKVOff + slot * C::kTileBytes;
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          mma_ts(tmem + 256 + t * 128, tmem + t * 128 + 64 + kk * 8,
+                 sdesc_sw128(va + kk * 2048, 16384, 1024), kIdescPV, (acc || kk > 0) ? 1u : 0u);
+      };
+      auto kv_wait = [&](uint32_t idx) {
+        return mbar_wait(&kv_full[idx % NS], (idx / NS) & 1u, abort_flag, kSiteKVFull);
+      };
+
+      bool ok = true;
+#pragma unroll
+      for (int t = 0; t < 2; ++t)
+        if (ok && n_t[t] > 0) ok = mbar_wait(&q_full[t], 0, abort_flag, kSiteQFull);
+      if (ok) ok = kv_wait(0);
+      if (ok) {
+        tc_fence_after();
+#pragma unroll
+        for (int t = 0; t < 2; ++t)
+          if (n_t[t] > 0) {
+            issue_qk(t, 0);
+            tc_commit(&s_full[t]);
+          }
+        tc_commit(&kv_empty[0]);
+      }
+      for (int j = 0; ok && j < n_max; ++j) {
+        const uint32_t iv = 2 * j + 1, ik = 2 * j + 2;
+        if (!kv_wait(iv)) { ok = false; break; }
+        tc_fence_after();
+        bool k_ready = false;
+#pragma unroll
+        for (int t = 0; t < 2; ++t) {
+          if (j >= n_t[t]) continue;
+          if (!mbar_wait(&p_full[t], j & 1, abort_flag, kSitePFull)) { ok = false; break; }
+          tc_fence_after();
+          issue_pv(t, iv % NS, j > 0);
+          if (j == n_t[t] - 1) {
+            tc_commit(&o_full[t]);
+          } else {
+            if (!k_ready) {
+              if (!kv_wait(ik)) { ok = false; break; }
+              tc_fence_after();
+              k_ready = true;
+            }
+            issue_qk(t, ik % NS);
+            tc_commit(&s_full[t]);
+          }
+        }
+        if (!ok) break;
+        tc_commit(&kv_empty[iv % NS]);
+        if (k_ready) tc_commit(&kv_empty[ik % NS]);
+      }
+      // Let this thread's MMAs finish before TMEM can be released.
+      tc_commit(mma_done);
+      mbar_wait_drain(mma_done, 0);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ softmax
+    regs_grow<kFwdRegsSoftmax>();
+    const int t = warp >> 2;
+    const int quad = warp & 3;
+    const int row = mb * 256 + t * 128 + quad * 32 + lane;
+    const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
+    const uint32_t t_s = tmem + lane_base + t * 128;
+    const uint32_t t_p = t_s + 64;
+    const uint32_t t_o = tmem + lane_base + 256 + t * 128;
+    const int n = n_t[t];
+    const bool mask_last = CAUSAL || (N & 127) != 0;
+    const int visible_end = CAUSAL ? min(row + 1, N) : N;   // keys [0, visible_end) are visible
+
+    float m_run = -INFINITY;   // running max, log2 units (scaled logits * log2 e)
+    float l_run = 0.f;         // running sum of 2^(t - m_run)
+    bool ok = n > 0;
+    for (int j = 0; ok && j < n; ++j) {
+      if (!mbar_wait(&s_full[t], j & 1, abort_flag, kSiteSFull)) { ok = false; break; }
+      tc_fence_after();
+      uint32_t r0[32], r1[32], r2[32], r3[32];
+      tmem_ld32(t_s + 0, r0);
+      tmem_ld32(t_s + 32, r1);
+      tmem_ld32(t_s + 64, r2);
+      tmem_ld32(t_s + 96, r3);
+      tmem_ld_wait(r0);
+      reg_fence(r1);
+      reg_fence(r2);
+      reg_fence(r3);
+
+      if (mask_last && j == n - 1) {
+        const int lim = visible_end - j * 128;   // columns [lim, 128) are masked
+        const uint32_t ninf = f2u(-INFINITY);
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          if (e >= lim) r0[e] = ninf;
+          if (32 + e >= lim) r1[e] = ninf;
+          if (64 + e >= lim) r2[e] = ninf;
+          if (96 + e >= lim) r3[e] = ninf;
+        }
+      }
+      float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
+#pragma unroll
+      for (int e = 0; e < 32; ++e) {
+        mx0 = fmaxf(mx0, u2f(r0[e]));
+        mx1 = fmaxf(mx1, u2f(r1[e]));
+        mx2 = fmaxf(mx2, u2f(r2[e]));
+        mx3 = fmaxf(mx3, u2f(r3[e]));
+      }
+      const float m_tile = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * scale_log2;
+      const float m_new = fmaxf(m_run, m_tile);
+      // Lazy rescale: keep the stale max unless the new one is more than 2^8 larger.
+      const bool need = m_new > m_run + 8.0f;
+      if (j > 0 && __any_sync(0xffffffffu, need)) {
+        const float f = need ? fast_exp2(m_run - m_new) : 1.0f;
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t o[32];
+          tmem_ld32(t_o + c * 32, o);
+          tmem_ld_wait(o);
+#pragma unroll
+          for (int e = 0; e < 32; ++e) o[e] = f2u(u2f(o[e]) * f);
+          tmem_st32(t_o + c * 32, o);
+        }
+      }
+      if (need) {
+        l_run *= fast_exp2(m_run - m_new);
+        m_run = m_new;
+      }
+      const float neg_m = -m_run;
+      float s0 = 0.f, s1 = 0.f;
+      // Exponentiate 32 columns at a time and store them as 16 packed bf16
+      // pairs right away, so at most 16 P words are live at once. The row sum
+      // adds the bf16-rounded values the PV MMA consumes, so numerator and
+      // denominator see the same weights (a one-hot row returns V exactly).
+      auto emit = [&](const uint32_t (&r)[32], uint32_t col) {
+        uint32_t pw[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          const float x0 = fast_exp2(fmaf(u2f(r[2 * e]), scale_log2, neg_m));
+          const float x1 = fast_exp2(fmaf(u2f(r[2 * e + 1]), scale_log2, neg_m));
+          const uint32_t pk = pack_bf16x2(x0, x1);
+          const float rounded = u2f(pk << 16) + u2f(pk & 0xFFFF0000u);
+          if (e & 1) s1 += rounded; else s0 += rounded;
+          pw[e] = pk;
+        }
+        tmem_st16(t_p + col, pw);
+      };
+      emit(r0, 0);
+      emit(r1, 16);
+      emit(r2, 32);
+      emit(r3, 48);
+      l_run += s0 + s1;
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(&p_full[t]);
+    }
+
+    if (ok) ok = mbar_wait(&o_full[t], 0, abort_flag, kSiteOFull);
+    if (ok) {
+      tc_fence_after();
+      const float inv_l = 1.0f / l_run;
+      __nv_bfloat16* orow = out + (static_cast<size_t>(bh) * N + row) * D;
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t o[32];
+        tmem_ld32(t_o + c * 32, o);
+        tmem_ld_wait(o);
+        uint32_t pk[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) pk[e] = pack_bf16x2(u2f(o[2 * e]) * inv_l, u2f(o[2 * e + 1]) * inv_l);
+        if (row < N) {
+          uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
+          dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+          dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+          dst[2] = make_uint4(pk[8], pk[9], pk[10], pk[11]);
+          dst[3] = make_uint4(pk[12], pk[13], pk[14], pk[15]);
+        }
+      }
+      if (row < N)
+        lse_out[static_cast<size_t>(bh) * N + row] = (m_run + __log2f(l_run)) * 0.69314718055994531f;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 9) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace attn

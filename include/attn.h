@@ -1,0 +1,122 @@
+/*
+ * attn.h: C ABI of the exact scaled-dot-product attention library for one
+ * NVIDIA B200 (sm_100a).
+ *
+ * Operation: hysenlabs.com, "FlashAttention: exakte Attention-Kernel fuer CUDA
+ * und ROCm", section "Die Schnittstellen von flash_attn_func bis KV-Cache".
+ * Every entry point computes
+ *
+ *     O = softmax(Q @ K^T * softmax_scale) @ V
+ *
+ * `causal` masks key j for query i when j > i. The bottom-right alignment
+ * (same page, section "Von 2.0 bis 2.7", release 2.1) is the same thing here,
+ * because queries and keys always have the same length N. K and V may have
+ * fewer heads than Q when Hq is divisible by Hkv (MQA/GQA, same interface
+ * section). Query head h reads KV head h / (Hq / Hkv).
+ *
+ * The method is exact, not an approximation (tokenwerk.de "FlashAttention",
+ * section "Was FlashAttention veraendert"). Results differ from a float64
+ * evaluation of the formula only by floating-point rounding. The N x N score
+ * matrix is never written to memory: tiles of Q, K and V are staged on chip,
+ * and a running row max and row sum normalise the output as it accumulates
+ * (unite.ai "Was ist FlashAttention?", five-stage map, stages 1-4).
+ *
+ * Conventions shared by all calls
+ *  - Tensors are contiguous, row-major [B, H, N, d] bfloat16 (d fastest).
+ *    lse and the workspace are float32.
+ *  - Every tensor pointer is a DEVICE pointer owned by the caller. It must
+ *    be 16-byte aligned and must not alias another argument. The library
+ *    allocates no memory and keeps no pointer after a call returns.
+ *  - Calls are asynchronous on `stream` (a cudaStream_t, may be 0), like a
+ *    kernel launch. They return after the launches are queued.
+ *  - Supported: d in {64, 128}; N >= 1 (any length; ragged tail tiles are
+ *    masked); B, Hq, Hkv >= 1; Hq % Hkv == 0; scale finite and > 0.
+ *    B == 0 or N == 0 is an empty problem: nothing is launched and ATTN_OK
+ *    is returned.
+ *  - Errors are return codes, never aborts. An argument error launches
+ *    nothing. The message of the last error on the calling thread is in
+ *    attn_get_last_error().
+ *  - There is no CPU fallback. Without a usable sm_100 device the calls
+ *    return ATTN_ERR_CUDA.
+ *  - Kernel waits are bounded. A kernel that stalls for two seconds on a
+ *    pipeline barrier records a timeout in a device status word and exits.
+ *    attn_check_status() reports it.
+ */
+#ifndef EXACT_ATTENTION_B200_ATTN_H_
+#define EXACT_ATTENTION_B200_ATTN_H_
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  ATTN_OK = 0,
+  ATTN_ERR_ARG = 1,          /* invalid argument (null/misaligned pointer, bad shape)   */
+  ATTN_ERR_UNSUPPORTED = 2,  /* valid but not built (head dim other than 64 or 128)     */
+  ATTN_ERR_CUDA = 3,         /* CUDA runtime/driver error, or no sm_100 device          */
+  ATTN_ERR_TIMEOUT = 4       /* a kernel gave up on a pipeline wait (see check_status)   */
+} attn_status;
+
+/* Opaque stream handle; pass a cudaStream_t (or 0 for the legacy default stream). */
+typedef void* attn_stream_t;
+
+/*
+ * attn_fwd: forward pass.
+ *   q    [B, Hq,  N, d] bf16, read
+ *   k, v [B, Hkv, N, d] bf16, read
+ *   o    [B, Hq,  N, d] bf16, written: softmax(q k^T * scale [causal]) v
+ *   lse  [B, Hq,  N]    f32,  written: natural-log logsumexp of the scaled,
+ *        masked logits of each query row, ln sum_j exp(scale * q_i . k_j).
+ *        (The pages do not define lse. This is the plainest definition
+ *        that the backward pass needs.)
+ *   scale: softmax_scale (for example 1/sqrt(d)); causal: 0 or 1.
+ */
+attn_status attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
+                     int B, int Hq, int Hkv, int N, int d, float scale, int causal,
+                     attn_stream_t stream);
+
+/*
+ * attn_bwd: recompute-based backward pass of attn_fwd.
+ *   q, k, v, o, lse: as passed to / returned by attn_fwd (read)
+ *   dO  [B, Hq,  N, d] bf16, read: gradient of the loss with respect to o
+ *   dq  [B, Hq,  N, d] bf16, written
+ *   dk, dv [B, Hkv, N, d] bf16, written. Under GQA each KV head's gradient
+ *        is the sum over the Hq/Hkv query heads that read it.
+ *   workspace: caller-owned device scratch of at least
+ *        attn_bwd_workspace_size(B, Hq, N, d) bytes, 16-byte aligned. Its
+ *        contents on entry are ignored, and it is overwritten.
+ * The pages do not write out the backward math. It is the exact gradient of
+ * the forward definition: dV = P^T dO, dS = P * (dP - rowsum(dO * O)) with
+ * dP = dO V^T, dQ = scale * dS K, dK = scale * dS^T Q. The P used is
+ * recomputed from q, k and lse, so no N x N matrix is stored. The result is
+ * deterministic: no atomics, the same bits on every run.
+ */
+attn_status attn_bwd(const void* q, const void* k, const void* v, const void* o,
+                     const float* lse, const void* dO, void* dq, void* dk, void* dv,
+                     void* workspace, size_t workspace_bytes, int B, int Hq, int Hkv, int N,
+                     int d, float scale, int causal, attn_stream_t stream);
+
+/* Bytes of workspace attn_bwd needs for this shape (0 for an empty problem). */
+size_t attn_bwd_workspace_size(int B, int Hq, int N, int d);
+
+/*
+ * Synchronises `stream`, then reads and clears the device status word.
+ * Returns ATTN_ERR_TIMEOUT if a kernel gave up on a wait since the last
+ * check, ATTN_ERR_CUDA on a CUDA error, and ATTN_OK otherwise.
+ */
+attn_status attn_check_status(attn_stream_t stream);
+
+/* Message of the last error on the calling thread ("" if none). The library
+ * owns the string. It stays valid until the next call on the same thread. */
+const char* attn_get_last_error(void);
+
+/* ABI version of this header: major * 100 + minor. */
+int attn_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* EXACT_ATTENTION_B200_ATTN_H_ */

@@ -1,0 +1,119 @@
+"""The C-ABI boundary on the CPU: the library loads, exports every symbol the
+header declares, and rejects bad arguments with status codes before touching
+a GPU. No compute call is made here (there is no GPU on the build machine)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import exact_attention_105_b200 as ea
+from exact_attention_105_b200 import build as eabuild
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "attn.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    eabuild.build()
+    return ea.load_library()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(attn_[a-z_0-9]+)\s*\(", text)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for required in ("attn_fwd", "attn_bwd", "attn_bwd_workspace_size", "attn_check_status",
+                     "attn_get_last_error"):
+        assert required in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+    assert set(declared_functions()) <= set(ea.SIGNATURES)
+    assert lib.attn_abi_version() == 100
+
+
+FAKE = 1 << 20          # aligned, non-null, but not device memory
+
+
+def fwd(lib, q=FAKE, k=FAKE, v=FAKE, o=FAKE, lse=FAKE, B=1, Hq=2, Hkv=1, N=128, d=64,
+        scale=0.125, causal=0):
+    return lib.attn_fwd(q, k, v, o, lse, B, Hq, Hkv, N, d, scale, causal, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(Hq=3, Hkv=2), ea.ATTN_ERR_ARG),          # GQA needs Hq % Hkv == 0
+    (dict(Hkv=0), ea.ATTN_ERR_ARG),
+    (dict(B=-1), ea.ATTN_ERR_ARG),
+    (dict(N=-5), ea.ATTN_ERR_ARG),
+    (dict(d=96), ea.ATTN_ERR_UNSUPPORTED),
+    (dict(d=256), ea.ATTN_ERR_UNSUPPORTED),
+    (dict(scale=0.0), ea.ATTN_ERR_ARG),
+    (dict(scale=float("nan")), ea.ATTN_ERR_ARG),
+    (dict(scale=float("inf")), ea.ATTN_ERR_ARG),
+    (dict(causal=2), ea.ATTN_ERR_ARG),
+    (dict(q=None), ea.ATTN_ERR_ARG),
+    (dict(lse=None), ea.ATTN_ERR_ARG),
+    (dict(k=FAKE + 8), ea.ATTN_ERR_ARG),           # TMA needs 16-byte alignment
+])
+def test_fwd_argument_errors(lib, kw, code):
+    assert fwd(lib, **kw) == code
+    assert lib.attn_get_last_error().decode() != ""
+
+
+def test_empty_problem_is_a_no_op(lib):
+    assert fwd(lib, B=0) == ea.ATTN_OK
+    assert fwd(lib, N=0) == ea.ATTN_OK
+    assert fwd(lib, q=None, k=None, v=None, o=None, lse=None, N=0) == ea.ATTN_OK
+
+
+def test_no_cpu_fallback_without_a_device(lib):
+    """Valid arguments on a machine without an sm_100 device: an error, never a CPU path."""
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    assert fwd(lib) == ea.ATTN_ERR_CUDA
+    assert "device" in lib.attn_get_last_error().decode().lower() or \
+        "cuda" in lib.attn_get_last_error().decode().lower()
+
+
+def bwd(lib, ws=FAKE, ws_bytes=1 << 30, B=1, Hq=2, Hkv=1, N=128, d=64, scale=0.125, causal=0,
+        **ptrs):
+    p = {n: FAKE for n in ("q", "k", "v", "o", "lse", "dO", "dq", "dk", "dv")}
+    p.update(ptrs)
+    return lib.attn_bwd(p["q"], p["k"], p["v"], p["o"], p["lse"], p["dO"], p["dq"], p["dk"],
+                        p["dv"], ws, ws_bytes, B, Hq, Hkv, N, d, scale, causal, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(Hq=4, Hkv=3), ea.ATTN_ERR_ARG),
+    (dict(d=32), ea.ATTN_ERR_UNSUPPORTED),
+    (dict(dO=None), ea.ATTN_ERR_ARG),
+    (dict(dv=FAKE + 4), ea.ATTN_ERR_ARG),
+    (dict(ws=None), ea.ATTN_ERR_ARG),
+    (dict(ws_bytes=16), ea.ATTN_ERR_ARG),          # smaller than attn_bwd_workspace_size
+    (dict(causal=-1), ea.ATTN_ERR_ARG),
+])
+def test_bwd_argument_errors(lib, kw, code):
+    assert bwd(lib, **kw) == code
+
+
+def test_workspace_size(lib):
+    assert lib.attn_bwd_workspace_size(0, 4, 128, 64) == 0
+    small = lib.attn_bwd_workspace_size(1, 1, 128, 64)
+    assert small >= 128 * 4                         # at least one fp32 per query row
+    assert lib.attn_bwd_workspace_size(8, 16, 2048, 128) >= 8 * 16 * 2048 * 4
+
+
+def test_binding_rejects_cpu_tensors():
+    import torch
+    q = torch.zeros(1, 1, 128, 64, dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="CUDA"):
+        ea.attn_fwd(q, q, q, o=q.clone(), lse=torch.zeros(1, 1, 128), causal=False)

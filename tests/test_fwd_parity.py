@@ -1,0 +1,119 @@
+"""GPU forward parity: the sm_100a kernel against the float64 oracle, on the
+same seeded bf16 inputs. Small and edge shapes are compared element by
+element over every output. The full-size workloads are compared on sampled
+rows that the oracle computes one at a time, plus properties that hold at
+any size.
+
+Tolerances: max|O - O_ref| <= 1e-2 and max|lse - lse_ref| <= 1e-3."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads
+from tests.gpu_helpers import (assert_fwd_close, gpu_fwd, max_err, naive_bf16_attention,
+                               sample_rows)
+
+pytestmark = pytest.mark.gpu
+
+
+def full_check(w):
+    q, k, v = workloads.make_inputs(w, with_grad_out=False)
+    o, lse = gpu_fwd(q, k, v, w.scale, w.causal)
+    o_ref, lse_ref = oracle.attention_forward(q, k, v, w.scale, w.causal)
+    return assert_fwd_close(o, lse, o_ref, lse_ref, w.name), (q, k, v, o, o_ref)
+
+
+def test_c1_tiny_noncausal():
+    full_check(workloads.C1)
+
+
+def test_c2_causal_d64():
+    full_check(workloads.C2)
+
+
+EDGE = []
+for d in (64, 128):
+    for causal in (False, True):
+        for n in (1, 17, 127, 128, 129, 255, 256, 257, 383, 520):
+            EDGE.append(workloads.small(f"edge_N{n}_d{d}_c{int(causal)}", 1, 2, 2, n, d, causal,
+                                        seed=n + d, backward=False))
+
+
+@pytest.mark.parametrize("w", EDGE, ids=lambda w: w.name)
+def test_ragged_and_tile_edge_lengths(w):
+    full_check(w)
+
+
+@pytest.mark.parametrize("hq,hkv", [(4, 1), (8, 2), (6, 3)])
+@pytest.mark.parametrize("causal", [False, True])
+def test_gqa_small(hq, hkv, causal):
+    w = workloads.small(f"gqa_{hq}_{hkv}_c{int(causal)}", 2, hq, hkv, 300, 128, causal, seed=hq * 10 + hkv,
+                        backward=False)
+    full_check(w)
+
+
+def test_error_within_twice_naive_bf16_baseline():
+    """Upstream methodology: the kernel's max error is at most twice that of a
+    plain bf16 attention measured against the same reference."""
+    w = workloads.small("naive_cmp", 2, 4, 4, 1024, 128, True, seed=11, backward=False)
+    (eo, _), (q, k, v, o, o_ref) = full_check(w)
+    naive = naive_bf16_attention(q, k, v, w.scale, w.causal).float().cpu().numpy()
+    e_naive, _ = max_err(naive, o_ref)
+    assert eo <= 2.0 * e_naive + 1e-6, (eo, e_naive)
+
+
+def test_large_logits_stress_small():
+    """Q scaled by 4 (exact in bf16): large logits exercise the lazy rescale."""
+    w = workloads.small("q4_small", 1, 4, 4, 1000, 128, True, q_mult=4.0, seed=5, backward=False)
+    full_check(w)
+
+
+@pytest.mark.parametrize("w", [workloads.C3_CAUSAL, workloads.C3_FULL, workloads.C3_STRESS,
+                               workloads.C4], ids=lambda w: w.name)
+def test_full_size_sampled_rows(w):
+    q, k, v = workloads.make_inputs(w, with_grad_out=False)
+    o, lse = gpu_fwd(q, k, v, w.scale, w.causal)
+    o_cpu = o.float().cpu().numpy()
+    lse_cpu = lse.cpu().numpy()
+    assert np.all(np.isfinite(o_cpu)) and np.all(np.isfinite(lse_cpu))
+    rng = np.random.default_rng(w.seed)
+    heads = {(0, 0), (w.B - 1, w.Hq - 1)}
+    while len(heads) < 6:
+        heads.add((int(rng.integers(w.B)), int(rng.integers(w.Hq))))
+    for b, h in sorted(heads):
+        rows = sample_rows(w.N, rng)
+        o_ref, lse_ref = oracle.attention_forward_rows(q, k, v, w.scale, w.causal, b, h, rows)
+        assert_fwd_close(o_cpu[b, h, rows], lse_cpu[b, h, rows], o_ref, lse_ref,
+                         f"{w.name} head ({b},{h})")
+    # Properties at any size: each output row is a convex combination of V
+    # rows (within bf16 rounding), and the lse is at least the causal-row
+    # lower bound max_j scale*q.k_j.
+    G = w.Hq // w.Hkv
+    vmax = v.float().amax(dim=2).repeat_interleave(G, dim=1).numpy()
+    vmin = v.float().amin(dim=2).repeat_interleave(G, dim=1).numpy()
+    assert np.all(o_cpu <= vmax[:, :, None, :] + 2e-2)
+    assert np.all(o_cpu >= vmin[:, :, None, :] - 2e-2)
+
+
+def test_repeat_runs_are_bitwise_identical():
+    w = workloads.small("det", 2, 4, 2, 700, 128, True, seed=3, backward=False)
+    q, k, v = workloads.make_inputs(w, with_grad_out=False)
+    o1, l1 = gpu_fwd(q, k, v, w.scale, True)
+    o2, l2 = gpu_fwd(q, k, v, w.scale, True)
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
+
+
+def test_non_default_scale():
+    w = workloads.small("scale", 1, 2, 2, 333, 64, False, seed=9, backward=False)
+    q, k, v = workloads.make_inputs(w, with_grad_out=False)
+    o, lse = gpu_fwd(q, k, v, 0.37, False)
+    o_ref, lse_ref = oracle.attention_forward(q, k, v, 0.37, False)
+    assert_fwd_close(o, lse, o_ref, lse_ref, "scale=0.37")
+
+
+def test_status_word_clean_after_runs():
+    import exact_attention_105_b200 as ea
+    ea.attn_check_status()
