@@ -32,7 +32,13 @@ SIGNATURES = {
     "attn_check_status": (_I, [_P]),
     "attn_get_last_error": (ctypes.c_char_p, []),
     "attn_abi_version": (_I, []),
+    "attn_profile_enable": (None, [_I]),
+    "attn_profile_reset": (None, []),
+    "attn_profile_read": (_I, [_I, ctypes.POINTER(ctypes.c_char_p), ctypes.POINTER(_I),
+                               ctypes.POINTER(ctypes.c_double)]),
 }
+
+PROFILED_KERNELS = ("fwd_kernel", "bwd_pre_kernel", "bwd_dkdv_kernel", "bwd_dq_kernel")
 
 _lib = None
 
@@ -149,6 +155,28 @@ def attn_bwd(q, k, v, o, lse, dO, dq=None, dk=None, dv=None, workspace=None, sca
                         workspace.numel() * workspace.element_size(),
                         B, Hq, Hkv, N, d, scale, int(bool(causal)), _stream_handle(stream)))
     return dq, dk, dv
+
+
+def profile_enable(on: bool = True):
+    """Turn per-kernel CUDA-event timing inside the library on or off."""
+    load_library().attn_profile_enable(int(bool(on)))
+
+
+def profile_reset():
+    load_library().attn_profile_reset()
+
+
+def profile_read():
+    """{kernel name: (launches, total milliseconds)} since the last reset."""
+    lib = load_library()
+    out = {}
+    for idx in range(len(PROFILED_KERNELS)):
+        name = ctypes.c_char_p()
+        n = ctypes.c_int()
+        ms = ctypes.c_double()
+        _check(lib.attn_profile_read(idx, ctypes.byref(name), ctypes.byref(n), ctypes.byref(ms)))
+        out[name.value.decode()] = (n.value, ms.value)
+    return out
 
 
 def attn_check_status(stream=None):

@@ -13,6 +13,7 @@
 #include <cstdio>
 #include <cstring>
 #include <mutex>
+#include <vector>
 
 #include "../../include/attn.h"
 #include "attn_bwd.cuh"
@@ -34,6 +35,56 @@ attn_status fail(attn_status code, const char* fmt, ...) {
 attn_status cuda_fail(cudaError_t e, const char* what) {
   return fail(ATTN_ERR_CUDA, "%s: %s (%s)", what, cudaGetErrorName(e), cudaGetErrorString(e));
 }
+
+// ---------------------------------------------------------------- profiling
+// Opt-in per-kernel timing: when enabled, every launch is bracketed by two
+// CUDA events recorded on the launch stream; attn_profile_read() sums the
+// elapsed times per kernel. Events come from a pool that grows on demand.
+enum ProfKernel { kProfFwd = 0, kProfBwdPre, kProfBwdDkdv, kProfBwdDq, kProfCount };
+const char* const kProfNames[kProfCount] = {"fwd_kernel", "bwd_pre_kernel", "bwd_dkdv_kernel",
+                                            "bwd_dq_kernel"};
+
+struct ProfState {
+  std::mutex mu;
+  bool on = false;
+  std::vector<cudaEvent_t> pool;
+  struct Pending { int kernel; cudaEvent_t a, b; };
+  std::vector<Pending> pending;
+  int launches[kProfCount] = {0, 0, 0, 0};
+  double total_ms[kProfCount] = {0, 0, 0, 0};
+};
+ProfState g_prof;
+
+cudaEvent_t prof_event() {
+  if (!g_prof.pool.empty()) {
+    cudaEvent_t e = g_prof.pool.back();
+    g_prof.pool.pop_back();
+    return e;
+  }
+  cudaEvent_t e = nullptr;
+  if (cudaEventCreate(&e) != cudaSuccess) return nullptr;
+  return e;
+}
+
+// Brackets one launch when profiling is on. Usage: ProfScope ps(kernel, s); launch; ps.end();
+struct ProfScope {
+  int kernel;
+  cudaStream_t stream;
+  cudaEvent_t a = nullptr, b = nullptr;
+  ProfScope(int k, cudaStream_t s) : kernel(k), stream(s) {
+    std::lock_guard<std::mutex> g(g_prof.mu);
+    if (!g_prof.on) return;
+    a = prof_event();
+    b = prof_event();
+    if (a && b) cudaEventRecord(a, stream);
+  }
+  void end() {
+    if (!a || !b) return;
+    cudaEventRecord(b, stream);
+    std::lock_guard<std::mutex> g(g_prof.mu);
+    g_prof.pending.push_back({kernel, a, b});
+  }
+};
 
 // ---------------------------------------------------------------- driver entry
 // cuTensorMapEncodeTiled is a driver API call; it is fetched through the
@@ -166,10 +217,73 @@ attn_status launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUten
                 launch_regs, attn::kFwdRegsLaunch);
   dim3 grid(B * Hq, (N + 255) / 256);
   const float scale_log2 = scale * 1.4426950408889634f;
+  ProfScope ps(kProfFwd, stream);
   kern<<<grid, Cfg::kThreads, Cfg::kSmemAlloc, stream>>>(
       mq, mk, mv, static_cast<__nv_bfloat16*>(o), lse, Hq, Hq / Hkv, N, scale_log2);
+  ps.end();
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "fwd kernel launch");
+  return ATTN_OK;
+}
+
+// One-time per-kernel setup: opt in to the dynamic shared memory size.
+template <typename Kern>
+cudaError_t set_smem_once(Kern kern, int bytes, std::once_flag& once, cudaError_t& err) {
+  std::call_once(once, [&] {
+    err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  });
+  return err;
+}
+
+struct BwdArgs {
+  CUtensorMap mq, mk, mv, mdo;
+  const void* o;
+  const float* lse;
+  const void* dO;
+  void *dq, *dk, *dv;
+  float *L, *Dv;
+  int B, Hq, Hkv, N;
+  float scale;
+};
+
+template <int D, bool CAUSAL>
+attn_status launch_bwd(const BwdArgs& a, cudaStream_t stream) {
+  using namespace attn;
+  const int Npad = pad128(a.N);
+  const int nblk = Npad / 128;
+  const int group = a.Hq / a.Hkv;
+  const float scale_log2 = a.scale * kLog2e;
+
+  const long long rows = static_cast<long long>(a.B) * a.Hq * Npad;
+  ProfScope p0(kProfBwdPre, stream);
+  bwd_pre_kernel<D><<<static_cast<unsigned>(rows / 32), 256, 0, stream>>>(
+      static_cast<const __nv_bfloat16*>(a.o), static_cast<const __nv_bfloat16*>(a.dO), a.lse,
+      a.L, a.Dv, a.N, Npad);
+  p0.end();
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "bwd preprocess launch");
+
+  static std::once_flag o1, o2;
+  static cudaError_t e1 = cudaSuccess, e2 = cudaSuccess;
+  auto k1 = bwd_dkdv_kernel<D, CAUSAL>;
+  auto k2 = bwd_dq_kernel<D, CAUSAL>;
+  if ((e = set_smem_once(k1, DkdvCfg<D>::kSmemAlloc, o1, e1)) != cudaSuccess)
+    return cuda_fail(e, "cudaFuncSetAttribute(dkdv)");
+  if ((e = set_smem_once(k2, DqCfg<D>::kSmemAlloc, o2, e2)) != cudaSuccess)
+    return cuda_fail(e, "cudaFuncSetAttribute(dq)");
+
+  ProfScope p1(kProfBwdDkdv, stream);
+  k1<<<dim3(a.B * a.Hkv, nblk), DkdvCfg<D>::kThreads, DkdvCfg<D>::kSmemAlloc, stream>>>(
+      a.mq, a.mk, a.mv, a.mdo, a.L, a.Dv, static_cast<__nv_bfloat16*>(a.dk),
+      static_cast<__nv_bfloat16*>(a.dv), a.Hq, group, a.N, Npad, scale_log2, a.scale);
+  p1.end();
+  if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "bwd dK/dV launch");
+  ProfScope p2(kProfBwdDq, stream);
+  k2<<<dim3(a.B * a.Hq, nblk), DqCfg<D>::kThreads, DqCfg<D>::kSmemAlloc, stream>>>(
+      a.mq, a.mk, a.mv, a.mdo, a.L, a.Dv, static_cast<__nv_bfloat16*>(a.dq), a.Hq, group, a.N,
+      Npad, scale_log2, a.scale);
+  p2.end();
+  if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "bwd dQ launch");
   return ATTN_OK;
 }
 
@@ -214,7 +328,9 @@ attn_status attn_fwd(const void* q, const void* k, const void* v, void* o, float
 size_t attn_bwd_workspace_size(int B, int Hq, int N, int d) {
   (void)d;
   if (B <= 0 || Hq <= 0 || N <= 0) return 0;
-  return static_cast<size_t>(B) * Hq * N * sizeof(float);
+  // lse * log2(e) and D = rowsum(dO * O), fp32, one row per query padded to
+  // a multiple of 128 per head.
+  return 2 * static_cast<size_t>(B) * Hq * attn::pad128(N) * sizeof(float);
 }
 
 attn_status attn_bwd(const void* q, const void* k, const void* v, const void* o,
@@ -239,8 +355,57 @@ attn_status attn_bwd(const void* q, const void* k, const void* v, const void* o,
   st = ensure_init();
   if (st != ATTN_OK) return st;
   if ((st = check_ptrs(ptrs, names, 10)) != ATTN_OK) return st;
-  (void)stream_;
-  return fail(ATTN_ERR_UNSUPPORTED, "attn_bwd: not built yet");
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+  CUtensorMap mq, mk, mv, mdo;
+  if ((st = make_map(&mq, q, d, N, B * Hq)) != ATTN_OK) return st;
+  if ((st = make_map(&mk, k, d, N, B * Hkv)) != ATTN_OK) return st;
+  if ((st = make_map(&mv, v, d, N, B * Hkv)) != ATTN_OK) return st;
+  if ((st = make_map(&mdo, dO, d, N, B * Hq)) != ATTN_OK) return st;
+  float* L = static_cast<float*>(workspace);
+  float* Dv = L + static_cast<size_t>(B) * Hq * attn::pad128(N);
+  BwdArgs a{mq, mk, mv, mdo, o, lse, dO, dq, dk, dv, L, Dv, B, Hq, Hkv, N, scale};
+  if (d == 64) return causal ? launch_bwd<64, true>(a, stream) : launch_bwd<64, false>(a, stream);
+  return causal ? launch_bwd<128, true>(a, stream) : launch_bwd<128, false>(a, stream);
+}
+
+void attn_profile_enable(int on) {
+  std::lock_guard<std::mutex> g(g_prof.mu);
+  g_prof.on = on != 0;
+}
+
+void attn_profile_reset(void) {
+  std::lock_guard<std::mutex> g(g_prof.mu);
+  for (auto& p : g_prof.pending) {
+    g_prof.pool.push_back(p.a);
+    g_prof.pool.push_back(p.b);
+  }
+  g_prof.pending.clear();
+  for (int k = 0; k < kProfCount; ++k) {
+    g_prof.launches[k] = 0;
+    g_prof.total_ms[k] = 0.0;
+  }
+}
+
+attn_status attn_profile_read(int kernel, const char** name, int* launches, double* total_ms) {
+  g_last_error[0] = '\0';
+  if (kernel < 0 || kernel >= kProfCount)
+    return fail(ATTN_ERR_ARG, "kernel index %d out of range [0, %d)", kernel, (int)kProfCount);
+  std::lock_guard<std::mutex> g(g_prof.mu);
+  for (auto& p : g_prof.pending) {
+    float ms = 0.f;
+    cudaError_t e = cudaEventSynchronize(p.b);
+    if (e == cudaSuccess) e = cudaEventElapsedTime(&ms, p.a, p.b);
+    if (e != cudaSuccess) return cuda_fail(e, "profile event");
+    g_prof.launches[p.kernel] += 1;
+    g_prof.total_ms[p.kernel] += ms;
+    g_prof.pool.push_back(p.a);
+    g_prof.pool.push_back(p.b);
+  }
+  g_prof.pending.clear();
+  if (name) *name = kProfNames[kernel];
+  if (launches) *launches = g_prof.launches[kernel];
+  if (total_ms) *total_ms = g_prof.total_ms[kernel];
+  return ATTN_OK;
 }
 
 attn_status attn_check_status(attn_stream_t stream_) {

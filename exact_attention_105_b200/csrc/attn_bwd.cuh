@@ -1,2 +1,670 @@
+// Backward kernels: dQ, dK, dV of O = softmax(Q K^T * scale [causal]) V.
+//
+// The pages give the forward formula only (hysenlabs.com "FlashAttention:
+// exakte Attention-Kernel fuer CUDA und ROCm", section "Die Schnittstellen
+// von flash_attn_func bis KV-Cache"), and list fwd+bwd among the upstream
+// kernels' features. The gradient computed here is the exact gradient of
+// that formula:
+//   P = exp(scale * Q K^T - lse)   (recomputed per tile from q, k and lse)
+//   dV = P^T dO,  dP = dO V^T,  dS = P * (dP - D),  D = rowsum(dO * O)
+//   dQ = scale * dS K,  dK = scale * dS^T Q
+// D = rowsum(dO * O) equals rowsum(P * dP) because O = P V.
+//
+// Three kernels, all deterministic (no atomics):
+//   bwd_pre_kernel   D and lse * log2(e), per query row, into the workspace,
+//                    padded to a multiple of 128 rows per head. Padding rows
+//                    get lse = +inf, so every P that involves them is 0.
+//   bwd_dkdv_kernel  one CTA per (batch, KV head, 128-key block). K_j and V_j
+//                    stay in shared memory. It loops over the 128-query blocks
+//                    of every query head in the GQA group (from the diagonal
+//                    when causal). Per block it computes S^T, dP^T, P^T, dS^T
+//                    and accumulates dV and dK in TMEM.
+//   bwd_dq_kernel    one CTA per (batch, query head, 128-query block). Q_i and
+//                    dO_i stay resident while K_j/V_j stream through a ring. Per
+//                    block it computes S, dP, P, dS and accumulates dQ in TMEM.
+// Warp roles in both main kernels (256 threads): warps 0-3 compute (thread r
+// owns TMEM lane r), warp 4 TMA producer, warp 5 TMEM allocator and MMA
+// issuer, warps 6-7 idle.
 #pragma once
+
 #include "sm100.cuh"
+
+namespace attn {
+
+constexpr float kLog2e = 1.4426950408889634f;
+
+__host__ __device__ inline int pad128(int n) { return (n + 127) & ~127; }
+
+// ------------------------------------------------------------------ preprocess
+// 8 lanes per query row, 4 rows per warp, 32 rows per 256-thread block. The
+// grid covers BH * Npad rows exactly (a multiple of 128), so every shuffle
+// group is fully populated.
+template <int D>
+__global__ void __launch_bounds__(256)
+bwd_pre_kernel(const __nv_bfloat16* __restrict__ o, const __nv_bfloat16* __restrict__ dO,
+               const float* __restrict__ lse, float* __restrict__ L, float* __restrict__ Dv, int N,
+               int Npad) {
+  const long long row = static_cast<long long>(blockIdx.x) * 32 + (threadIdx.x >> 3);
+  const int sub = threadIdx.x & 7;
+  const long long bh = row / Npad;
+  const int n = static_cast<int>(row - bh * Npad);
+  float acc = 0.f;
+  if (n < N) {
+    constexpr int kPer = D / 8;  // elements per lane: 16 (D=128) or 8 (D=64)
+    const size_t base = (static_cast<size_t>(bh) * N + n) * D + sub * kPer;
+    const uint4* po = reinterpret_cast<const uint4*>(o + base);
+    const uint4* pd = reinterpret_cast<const uint4*>(dO + base);
+#pragma unroll
+    for (int v = 0; v < kPer / 8; ++v) {
+      const uint4 a = po[v], b = pd[v];
+      const uint32_t aw[4] = {a.x, a.y, a.z, a.w}, bw[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        acc = fmaf(u2f(aw[e] << 16), u2f(bw[e] << 16), acc);
+        acc = fmaf(u2f(aw[e] & 0xFFFF0000u), u2f(bw[e] & 0xFFFF0000u), acc);
+      }
+    }
+  }
+  acc += __shfl_xor_sync(0xffffffffu, acc, 4);
+  acc += __shfl_xor_sync(0xffffffffu, acc, 2);
+  acc += __shfl_xor_sync(0xffffffffu, acc, 1);
+  if (sub == 0) {
+    L[row] = (n < N) ? lse[static_cast<size_t>(bh) * N + n] * kLog2e : INFINITY;
+    Dv[row] = (n < N) ? acc : 0.f;
+  }
+}
+
+// ------------------------------------------------------------------ shared bits
+enum BwdSite : int {
+  kSiteBKV = 0x11, kSiteBLoadFull = 0x12, kSiteBLoadEmpty = 0x13, kSiteBS = 0x14,
+  kSiteBDP = 0x15, kSiteBP = 0x16, kSiteBDS = 0x17, kSiteBAcc = 0x18, kSiteBSFree = 0x19
+};
+
+// Loads a 128-column fp32 row block from TMEM into four 32-register blocks.
+__device__ __forceinline__ void tmem_ld128(uint32_t taddr, uint32_t (&r0)[32], uint32_t (&r1)[32],
+                                           uint32_t (&r2)[32], uint32_t (&r3)[32]) {
+  tmem_ld32(taddr + 0, r0);
+  tmem_ld32(taddr + 32, r1);
+  tmem_ld32(taddr + 64, r2);
+  tmem_ld32(taddr + 96, r3);
+  tmem_ld_wait(r0);
+  reg_fence(r1);
+  reg_fence(r2);
+  reg_fence(r3);
+}
+
+// dS = P * (dP - Dcol) for 32 columns, P given as 16 packed bf16 pairs;
+// writes 16 packed bf16 pairs of dS. `dsub(e)` gives the D value of column e.
+template <typename DSub>
+__device__ __forceinline__ void ds_block(const uint32_t* pw, const uint32_t (&dp)[32],
+                                         uint32_t* out, DSub dsub) {
+#pragma unroll
+  for (int e = 0; e < 16; ++e) {
+    const float p0 = u2f(pw[e] << 16), p1 = u2f(pw[e] & 0xFFFF0000u);
+    const float a = p0 * (u2f(dp[2 * e]) - dsub(2 * e));
+    const float b = p1 * (u2f(dp[2 * e + 1]) - dsub(2 * e + 1));
+    out[e] = pack_bf16x2(a, b);
+  }
+}
+
+// Epilogue helper: one 128 x D fp32 accumulator row (this thread's lane) ->
+// bf16 * mul, stored to `dst` when `valid`.
+template <int D>
+__device__ __forceinline__ void store_acc_row(uint32_t t_acc, __nv_bfloat16* dst, float mul,
+                                              bool valid) {
+#pragma unroll
+  for (int c = 0; c < D / 32; ++c) {
+    uint32_t a[32];
+    tmem_ld32(t_acc + c * 32, a);
+    tmem_ld_wait(a);
+    uint32_t pk[16];
+#pragma unroll
+    for (int e = 0; e < 16; ++e) pk[e] = pack_bf16x2(u2f(a[2 * e]) * mul, u2f(a[2 * e + 1]) * mul);
+    if (valid) {
+      uint4* p = reinterpret_cast<uint4*>(dst + c * 32);
+      p[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+      p[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+      p[2] = make_uint4(pk[8], pk[9], pk[10], pk[11]);
+      p[3] = make_uint4(pk[12], pk[13], pk[14], pk[15]);
+    }
+  }
+}
+
+// ------------------------------------------------------------------ dK / dV
+template <int D>
+struct DkdvCfg {
+  static constexpr int kTile = 128 * D * 2;
+  static constexpr int kStages = (D == 128) ? 2 : 4;     // (Q_i, dO_i, L_i, D_i) stages
+  static constexpr int kKOff = 0;
+  static constexpr int kVOff = kTile;
+  static constexpr int kStageOff = 2 * kTile;
+  static constexpr int kStageBytes = 2 * kTile + 1024;   // Q, dO, 128 L floats, 128 D floats
+  static constexpr int kBarOff = kStageOff + kStages * kStageBytes;
+  // kv_full ld_full[S] ld_empty[S] s_full dp_full p_full ds_full acc_done mma_done
+  static constexpr int kNumBars = 1 + 2 * kStages + 6;
+  static constexpr int kMiscOff = kBarOff + kNumBars * 8;
+  static constexpr int kBytes = kMiscOff + 16;
+  static constexpr int kSmemAlloc = kBytes + 1024;
+  static constexpr int kThreads = 256;
+};
+
+template <int D, bool CAUSAL>
+__global__ void __launch_bounds__(256, 1)
+bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+                const float* __restrict__ Lws, const float* __restrict__ Dws,
+                __nv_bfloat16* __restrict__ dk, __nv_bfloat16* __restrict__ dv, int Hq, int group,
+                int N, int Npad, float scale_log2, float scale) {
+  using C = DkdvCfg<D>;
+  constexpr int NS = C::kStages;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  const uint32_t sbase = smem_u32(smem);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kBarOff);
+  uint64_t* kv_full = bars;
+  uint64_t* ld_full = kv_full + 1;
+  uint64_t* ld_empty = ld_full + NS;
+  uint64_t* s_full = ld_empty + NS;
+  uint64_t* dp_full = s_full + 1;
+  uint64_t* p_full = dp_full + 1;
+  uint64_t* ds_full = p_full + 1;
+  uint64_t* acc_done = ds_full + 1;
+  uint64_t* mma_done = acc_done + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kMiscOff);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kMiscOff + 4);
+
+  const int warp = warp_id(), lane = lane_id();
+  const int Hkv = Hq / group;
+  const int bh_kv = blockIdx.x;
+  const int b = bh_kv / Hkv;
+  const int hkv = bh_kv - b * Hkv;
+  const int j = blockIdx.y;                   // KV block: low j has the most causal work
+  const int nq = (N + 127) >> 7;
+  const int i_start = CAUSAL ? j : 0;
+  const int per_head = nq - i_start;
+  const int n_steps = group * per_head;       // >= 1
+
+  if (threadIdx.x == 0) {
+    mbar_init(kv_full, 1);
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(&ld_full[s], 1);
+      mbar_init(&ld_empty[s], 1);
+    }
+    mbar_init(s_full, 1);
+    mbar_init(dp_full, 1);
+    mbar_init(p_full, 128);
+    mbar_init(ds_full, 128);
+    mbar_init(acc_done, 1);
+    mbar_init(mma_done, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 5) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  auto step_head = [&](int s, int& i, int& bh_q) {
+    const int g = s / per_head;
+    i = i_start + (s - g * per_head);
+    bh_q = b * Hq + hkv * group + g;
+  };
+
+  if (warp == 4) {
+    if (lane == 0) {
+      // -------------------------------------------------------- producer
+      tma_prefetch_desc(&tm_q);
+      tma_prefetch_desc(&tm_k);
+      tma_prefetch_desc(&tm_v);
+      tma_prefetch_desc(&tm_do);
+      mbar_expect_tx(kv_full, 2 * C::kTile);
+#pragma unroll
+      for (int a = 0; a < D / 64; ++a) {
+        tma_load_3d(smem + C::kKOff + a * 16384, &tm_k, kv_full, a * 64, j * 128, bh_kv);
+        tma_load_3d(smem + C::kVOff + a * 16384, &tm_v, kv_full, a * 64, j * 128, bh_kv);
+      }
+      int issued = 0;
+      for (int s = 0; s < n_steps; ++s) {
+        const int st = s % NS, round = s / NS;
+        if (round > 0 && !mbar_wait(&ld_empty[st], (round - 1) & 1, abort_flag, kSiteBLoadEmpty)) break;
+        int i, bh_q;
+        step_head(s, i, bh_q);
+        uint8_t* stage = smem + C::kStageOff + st * C::kStageBytes;
+        mbar_expect_tx(&ld_full[st], 2 * C::kTile + 1024);
+#pragma unroll
+        for (int a = 0; a < D / 64; ++a) {
+          tma_load_3d(stage + a * 16384, &tm_q, &ld_full[st], a * 64, i * 128, bh_q);
+          tma_load_3d(stage + C::kTile + a * 16384, &tm_do, &ld_full[st], a * 64, i * 128, bh_q);
+        }
+        const size_t off = static_cast<size_t>(bh_q) * Npad + i * 128;
+        bulk_load(stage + 2 * C::kTile, Lws + off, 512, &ld_full[st]);
+        bulk_load(stage + 2 * C::kTile + 512, Dws + off, 512, &ld_full[st]);
+        ++issued;
+      }
+      mbar_wait_drain(kv_full, 0);
+      const int first = issued > NS ? issued - NS : 0;
+      for (int s = first; s < issued; ++s) mbar_wait_drain(&ld_full[s % NS], (s / NS) & 1);
+    }
+  } else if (warp == 5) {
+    if (lane == 0) {
+      // -------------------------------------------------------- MMA issuer
+      constexpr uint32_t kIdescSS = idesc_bf16_f32(128, 128, 0, 0);
+      constexpr uint32_t kIdescAcc = idesc_bf16_f32(128, D, 0, 1);
+      auto stage_addr = [&](int s) { return sbase + C::kStageOff + (s % NS) * C::kStageBytes; };
+      // dst(tmem) = A_kmajor(smem tile) * B_kmajor(smem tile)^T, K = D
+      auto mma_tile_kk = [&](uint32_t dst, uint32_t a, uint32_t bt) {
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+          mma_ss(dst, sdesc_sw128(a + off, 16, 1024), sdesc_sw128(bt + off, 16, 1024), kIdescSS,
+                 kk > 0 ? 1u : 0u);
+        }
+      };
+      // acc(tmem) += A(tmem, 128 x 128 bf16) * B(smem tile, MN-major), K = 128
+      auto mma_acc = [&](uint32_t acc, uint32_t a_tmem, uint32_t b, bool accumulate) {
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          mma_ts(acc, a_tmem + kk * 8, sdesc_sw128(b + kk * 2048, 16384, 1024), kIdescAcc,
+                 (accumulate || kk > 0) ? 1u : 0u);
+      };
+      bool ok = mbar_wait(kv_full, 0, abort_flag, kSiteBKV) &&
+                mbar_wait(&ld_full[0], 0, abort_flag, kSiteBLoadFull);
+      if (ok) {
+        tc_fence_after();
+        mma_tile_kk(tmem + 0, sbase + C::kKOff, stage_addr(0));                 // S^T(0)
+        tc_commit(s_full);
+        mma_tile_kk(tmem + 128, sbase + C::kVOff, stage_addr(0) + C::kTile);    // dP^T(0)
+        tc_commit(dp_full);
+      }
+      for (int s = 0; ok && s < n_steps; ++s) {
+        const uint32_t sa = stage_addr(s);
+        if (!mbar_wait(p_full, s & 1, abort_flag, kSiteBP)) { ok = false; break; }
+        tc_fence_after();
+        mma_acc(tmem + 256, tmem + 64, sa + C::kTile, s > 0);                     // dV += P^T dO
+        const bool more = s + 1 < n_steps;
+        if (more) {
+          if (!mbar_wait(&ld_full[(s + 1) % NS], ((s + 1) / NS) & 1, abort_flag, kSiteBLoadFull)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          mma_tile_kk(tmem + 0, sbase + C::kKOff, stage_addr(s + 1));            // S^T(s+1)
+          tc_commit(s_full);
+        }
+        if (!mbar_wait(ds_full, s & 1, abort_flag, kSiteBDS)) { ok = false; break; }
+        tc_fence_after();
+        mma_acc(tmem + 384, tmem + 192, sa, s > 0);                               // dK += dS^T Q
+        tc_commit(&ld_empty[s % NS]);
+        if (more) {
+          mma_tile_kk(tmem + 128, sbase + C::kVOff, stage_addr(s + 1) + C::kTile); // dP^T(s+1)
+          tc_commit(dp_full);
+        }
+      }
+      if (ok) tc_commit(acc_done);
+      tc_commit(mma_done);
+      mbar_wait_drain(mma_done, 0);
+    }
+    __syncwarp();
+  } else if (warp < 4) {
+    // ---------------------------------------------------------- compute
+    const int t = warp * 32 + lane;                   // key row within the block
+    const int key = j * 128 + t;
+    const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+    const uint32_t t_s = tmem + lane_base;            // S^T, P^T at +64
+    const uint32_t t_dp = tmem + lane_base + 128;     // dP^T, dS^T at +64
+    bool ok = true;
+    for (int s = 0; ok && s < n_steps; ++s) {
+      int i, bh_q;
+      step_head(s, i, bh_q);
+      const int st = s % NS;
+      const float* Ls = reinterpret_cast<const float*>(smem + C::kStageOff + st * C::kStageBytes + 2 * C::kTile);
+      const float* Ds = Ls + 128;
+      if (!mbar_wait(&ld_full[st], (s / NS) & 1, abort_flag, kSiteBLoadFull) ||
+          !mbar_wait(s_full, s & 1, abort_flag, kSiteBS)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      uint32_t r0[32], r1[32], r2[32], r3[32];
+      tmem_ld128(t_s, r0, r1, r2, r3);
+      const bool diag = CAUSAL && (i == j);           // key t sees query c only if c >= t
+      uint32_t pw[64];
+      auto p_block = [&](const uint32_t (&r)[32], int c0) {
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          const int c = c0 + 2 * e;
+          float p0 = fast_exp2(fmaf(u2f(r[2 * e]), scale_log2, -Ls[c]));
+          float p1 = fast_exp2(fmaf(u2f(r[2 * e + 1]), scale_log2, -Ls[c + 1]));
+          if (diag) {
+            if (c < t) p0 = 0.f;
+            if (c + 1 < t) p1 = 0.f;
+          }
+          pw[c0 / 2 + e] = pack_bf16x2(p0, p1);
+        }
+      };
+      p_block(r0, 0);
+      p_block(r1, 32);
+      p_block(r2, 64);
+      p_block(r3, 96);
+#pragma unroll
+      for (int c = 0; c < 4; ++c) tmem_st16(t_s + 64 + 16 * c, &pw[16 * c]);
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(p_full);
+
+      if (!mbar_wait(dp_full, s & 1, abort_flag, kSiteBDP)) { ok = false; break; }
+      tc_fence_after();
+      // dS^T goes to dP^T columns [64,128): read those dP^T columns first.
+      uint32_t d2[32], d3[32];
+      tmem_ld32(t_dp + 64, d2);
+      tmem_ld32(t_dp + 96, d3);
+      tmem_ld_wait(d2);
+      reg_fence(d3);
+      uint32_t ds[16];
+      {
+        uint32_t d0[32];
+        tmem_ld32(t_dp + 0, d0);
+        tmem_ld_wait(d0);
+        ds_block(&pw[0], d0, ds, [&](int e) { return Ds[e]; });
+        tmem_st16(t_dp + 64, ds);
+      }
+      {
+        uint32_t d1[32];
+        tmem_ld32(t_dp + 32, d1);
+        tmem_ld_wait(d1);
+        ds_block(&pw[16], d1, ds, [&](int e) { return Ds[32 + e]; });
+        tmem_st16(t_dp + 80, ds);
+      }
+      ds_block(&pw[32], d2, ds, [&](int e) { return Ds[64 + e]; });
+      tmem_st16(t_dp + 96, ds);
+      ds_block(&pw[48], d3, ds, [&](int e) { return Ds[96 + e]; });
+      tmem_st16(t_dp + 112, ds);
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(ds_full);
+    }
+    if (ok) ok = mbar_wait(acc_done, 0, abort_flag, kSiteBAcc);
+    if (ok) {
+      tc_fence_after();
+      const bool valid = key < N;
+      const size_t row_off = (static_cast<size_t>(bh_kv) * N + (valid ? key : 0)) * D;
+      store_acc_row<D>(tmem + lane_base + 256, dv + row_off, 1.0f, valid);
+      store_acc_row<D>(tmem + lane_base + 384, dk + row_off, scale, valid);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 5) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// ------------------------------------------------------------------ dQ
+template <int D>
+struct DqCfg {
+  static constexpr int kTile = 128 * D * 2;
+  static constexpr int kStages = (D == 128) ? 4 : 6;     // K/V ring slots
+  static constexpr int kQOff = 0;
+  static constexpr int kDOOff = kTile;
+  static constexpr int kKVOff = 2 * kTile;
+  static constexpr int kBarOff = kKVOff + kStages * kTile;
+  // qd_full kv_full[S] kv_empty[S] s_full s_free dp_full ds_full acc_done mma_done
+  static constexpr int kNumBars = 1 + 2 * kStages + 6;
+  static constexpr int kMiscOff = kBarOff + kNumBars * 8;
+  static constexpr int kBytes = kMiscOff + 16;
+  static constexpr int kSmemAlloc = kBytes + 1024;
+  static constexpr int kThreads = 256;
+};
+
+template <int D, bool CAUSAL>
+__global__ void __launch_bounds__(256, 1)
+bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+              const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+              const float* __restrict__ Lws, const float* __restrict__ Dws,
+              __nv_bfloat16* __restrict__ dq, int Hq, int group, int N, int Npad, float scale_log2,
+              float scale) {
+  using C = DqCfg<D>;
+  constexpr int NS = C::kStages;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  const uint32_t sbase = smem_u32(smem);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kBarOff);
+  uint64_t* qd_full = bars;
+  uint64_t* kv_full = qd_full + 1;
+  uint64_t* kv_empty = kv_full + NS;
+  uint64_t* s_full = kv_empty + NS;
+  uint64_t* s_free = s_full + 1;
+  uint64_t* dp_full = s_free + 1;
+  uint64_t* ds_full = dp_full + 1;
+  uint64_t* acc_done = ds_full + 1;
+  uint64_t* mma_done = acc_done + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kMiscOff);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kMiscOff + 4);
+
+  const int warp = warp_id(), lane = lane_id();
+  const int bh = blockIdx.x;
+  const int b = bh / Hq;
+  const int hq = bh - b * Hq;
+  const int bh_kv = b * (Hq / group) + hq / group;
+  const int nkv = (N + 127) >> 7;
+  const int i = gridDim.y - 1 - blockIdx.y;  // heaviest causal query blocks first
+  const int n = CAUSAL ? min(i + 1, nkv) : nkv;
+
+  if (threadIdx.x == 0) {
+    mbar_init(qd_full, 1);
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(&kv_full[s], 1);
+      mbar_init(&kv_empty[s], 1);
+    }
+    mbar_init(s_full, 1);
+    mbar_init(s_free, 128);
+    mbar_init(dp_full, 1);
+    mbar_init(ds_full, 128);
+    mbar_init(acc_done, 1);
+    mbar_init(mma_done, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 5) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 4) {
+    if (lane == 0) {
+      // -------------------------------------------------------- producer
+      tma_prefetch_desc(&tm_q);
+      tma_prefetch_desc(&tm_k);
+      tma_prefetch_desc(&tm_v);
+      tma_prefetch_desc(&tm_do);
+      mbar_expect_tx(qd_full, 2 * C::kTile);
+#pragma unroll
+      for (int a = 0; a < D / 64; ++a) {
+        tma_load_3d(smem + C::kQOff + a * 16384, &tm_q, qd_full, a * 64, i * 128, bh);
+        tma_load_3d(smem + C::kDOOff + a * 16384, &tm_do, qd_full, a * 64, i * 128, bh);
+      }
+      uint32_t issued = 0;
+      bool ok = true;
+      for (int jj = 0; jj < n && ok; ++jj) {
+        for (int w = 0; w < 2; ++w) {
+          const uint32_t s = issued % NS, round = issued / NS;
+          if (round > 0 && !mbar_wait(&kv_empty[s], (round - 1) & 1u, abort_flag, kSiteBLoadEmpty)) {
+            ok = false;
+            break;
+          }
+          mbar_expect_tx(&kv_full[s], C::kTile);
+#pragma unroll
+          for (int a = 0; a < D / 64; ++a)
+            tma_load_3d(smem + C::kKVOff + s * C::kTile + a * 16384, w ? &tm_v : &tm_k, &kv_full[s],
+                        a * 64, jj * 128, bh_kv);
+          ++issued;
+        }
+      }
+      mbar_wait_drain(qd_full, 0);
+      const uint32_t first = issued > (uint32_t)NS ? issued - NS : 0u;
+      for (uint32_t x = first; x < issued; ++x) mbar_wait_drain(&kv_full[x % NS], (x / NS) & 1u);
+    }
+  } else if (warp == 5) {
+    if (lane == 0) {
+      // -------------------------------------------------------- MMA issuer
+      constexpr uint32_t kIdescSS = idesc_bf16_f32(128, 128, 0, 0);
+      constexpr uint32_t kIdescAcc = idesc_bf16_f32(128, D, 0, 1);
+      auto slot = [&](uint32_t idx) { return sbase + C::kKVOff + (idx % NS) * C::kTile; };
+      auto kv_wait = [&](uint32_t idx) {
+        return mbar_wait(&kv_full[idx % NS], (idx / NS) & 1u, abort_flag, kSiteBKV);
+      };
+      auto mma_tile_kk = [&](uint32_t dst, uint32_t a, uint32_t bt) {
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+          mma_ss(dst, sdesc_sw128(a + off, 16, 1024), sdesc_sw128(bt + off, 16, 1024), kIdescSS,
+                 kk > 0 ? 1u : 0u);
+        }
+      };
+      bool ok = mbar_wait(qd_full, 0, abort_flag, kSiteBLoadFull) && kv_wait(0);
+      if (ok) {
+        tc_fence_after();
+        mma_tile_kk(tmem + 0, sbase + C::kQOff, slot(0));        // S(0) = Q K_0^T
+        tc_commit(s_full);
+        ok = kv_wait(1);
+      }
+      if (ok) {
+        tc_fence_after();
+        mma_tile_kk(tmem + 128, sbase + C::kDOOff, slot(1));     // dP(0) = dO V_0^T
+        tc_commit(dp_full);
+      }
+      for (int jj = 0; ok && jj < n; ++jj) {
+        const uint32_t ik = 2 * jj, iv = 2 * jj + 1;
+        const bool more = jj + 1 < n;
+        if (more) {
+          if (!mbar_wait(s_free, jj & 1, abort_flag, kSiteBSFree) || !kv_wait(ik + 2)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          mma_tile_kk(tmem + 0, sbase + C::kQOff, slot(ik + 2));  // S(j+1)
+          tc_commit(s_full);
+        }
+        if (!mbar_wait(ds_full, jj & 1, abort_flag, kSiteBDS)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t kb = slot(ik);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)                           // dQ += dS K_j
+          mma_ts(tmem + 256, tmem + 192 + kk * 8, sdesc_sw128(kb + kk * 2048, 16384, 1024),
+                 kIdescAcc, (jj > 0 || kk > 0) ? 1u : 0u);
+        tc_commit(&kv_empty[ik % NS]);
+        tc_commit(&kv_empty[iv % NS]);
+        if (more) {
+          if (!kv_wait(iv + 2)) { ok = false; break; }
+          tc_fence_after();
+          mma_tile_kk(tmem + 128, sbase + C::kDOOff, slot(iv + 2)); // dP(j+1)
+          tc_commit(dp_full);
+        }
+      }
+      if (ok) tc_commit(acc_done);
+      tc_commit(mma_done);
+      mbar_wait_drain(mma_done, 0);
+    }
+    __syncwarp();
+  } else if (warp < 4) {
+    // ---------------------------------------------------------- compute
+    const int t = warp * 32 + lane;                  // query row within the block
+    const int row = i * 128 + t;
+    const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+    const uint32_t t_s = tmem + lane_base;
+    const uint32_t t_dp = tmem + lane_base + 128;
+    const size_t ws = static_cast<size_t>(bh) * Npad + row;   // row < Npad always
+    const float Lr = Lws[ws];                                 // +inf on padding rows
+    const float Dr = Dws[ws];
+    bool ok = true;
+    for (int jj = 0; ok && jj < n; ++jj) {
+      if (!mbar_wait(s_full, jj & 1, abort_flag, kSiteBS)) { ok = false; break; }
+      tc_fence_after();
+      uint32_t r0[32], r1[32], r2[32], r3[32];
+      tmem_ld128(t_s, r0, r1, r2, r3);
+      tc_fence_before();
+      mbar_arrive(s_free);
+      const bool diag = CAUSAL && (jj == i);          // query t sees key c only if c <= t
+      // Keys past N (zero rows from the TMA fill) get P = 0 explicitly, so an
+      // extreme lse can never turn 0 * exp2(-lse) into a NaN.
+      const int klim = (jj == nkv - 1) ? N - jj * 128 : 128;
+      uint32_t pw[64];
+      auto p_block = [&](const uint32_t (&r)[32], int c0) {
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          const int c = c0 + 2 * e;
+          float p0 = fast_exp2(fmaf(u2f(r[2 * e]), scale_log2, -Lr));
+          float p1 = fast_exp2(fmaf(u2f(r[2 * e + 1]), scale_log2, -Lr));
+          if (diag) {
+            if (c > t) p0 = 0.f;
+            if (c + 1 > t) p1 = 0.f;
+          }
+          if (c >= klim) p0 = 0.f;
+          if (c + 1 >= klim) p1 = 0.f;
+          pw[c0 / 2 + e] = pack_bf16x2(p0, p1);
+        }
+      };
+      p_block(r0, 0);
+      p_block(r1, 32);
+      p_block(r2, 64);
+      p_block(r3, 96);
+
+      if (!mbar_wait(dp_full, jj & 1, abort_flag, kSiteBDP)) { ok = false; break; }
+      tc_fence_after();
+      uint32_t d2[32], d3[32];
+      tmem_ld32(t_dp + 64, d2);
+      tmem_ld32(t_dp + 96, d3);
+      tmem_ld_wait(d2);
+      reg_fence(d3);
+      uint32_t ds[16];
+      auto dsub = [&](int) { return Dr; };
+      {
+        uint32_t d0[32];
+        tmem_ld32(t_dp + 0, d0);
+        tmem_ld_wait(d0);
+        ds_block(&pw[0], d0, ds, dsub);
+        tmem_st16(t_dp + 64, ds);
+      }
+      {
+        uint32_t d1[32];
+        tmem_ld32(t_dp + 32, d1);
+        tmem_ld_wait(d1);
+        ds_block(&pw[16], d1, ds, dsub);
+        tmem_st16(t_dp + 80, ds);
+      }
+      ds_block(&pw[32], d2, ds, dsub);
+      tmem_st16(t_dp + 96, ds);
+      ds_block(&pw[48], d3, ds, dsub);
+      tmem_st16(t_dp + 112, ds);
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(ds_full);
+    }
+    if (ok) ok = mbar_wait(acc_done, 0, abort_flag, kSiteBAcc);
+    if (ok) {
+      tc_fence_after();
+      const bool valid = row < N;
+      store_acc_row<D>(tmem + lane_base + 256, dq + (static_cast<size_t>(bh) * N + (valid ? row : 0)) * D,
+                       scale, valid);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 5) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace attn

@@ -60,23 +60,8 @@ struct FwdCfg {
 // Wait-site ids reported in the status word when a wait times out.
 enum FwdSite : int {
   kSiteQFull = 1, kSiteKVFull = 2, kSiteKVEmpty = 3, kSiteSFull = 4, kSitePFull = 5,
-  kSiteOFull = 6, kSiteDrain = 7
+  kSiteOFull = 6
 };
-
-// Bounded wait that ignores the abort flag: used only to let this thread's
-// own in-flight asynchronous copies / MMAs land before the CTA exits.
-__device__ __forceinline__ void mbar_wait_drain(uint64_t* bar, uint32_t parity) {
-  const unsigned long long t0 = global_ns();
-  while (!mbar_try_wait(bar, parity)) {
-    if (global_ns() - t0 > kWaitTimeoutNs) {
-      atomicCAS(&g_attn_device_status, 0, kDevTimeout | (kSiteDrain << 8));
-      return;
-    }
-  }
-}
-
-__device__ __forceinline__ float u2f(uint32_t x) { return __uint_as_float(x); }
-__device__ __forceinline__ uint32_t f2u(float x) { return __float_as_uint(x); }
 
 // Register split: launched at kFwdRegsLaunch per thread (384 threads fill the
 // 64K register file); warpgroup 2 (producer, MMA, idle) drops to
@@ -280,7 +265,8 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
     const int visible_end = CAUSAL ? min(row + 1, N) : N;   // keys [0, visible_end) are visible
 
     float m_run = -INFINITY;   // running max, log2 units (scaled logits * log2 e)
-    float l_run = 0.f;         // running sum of 2^(t - m_run)
+    float l_run = 0.f;         // running sum of 2^(t - m_run), unrounded (for lse)
+    float l_mma = 0.f;         // running sum of the bf16-rounded P fed to the MMA (for O)
     bool ok = n > 0;
     for (int j = 0; ok && j < n; ++j) {
       if (!mbar_wait(&s_full[t], j & 1, abort_flag, kSiteSFull)) { ok = false; break; }
@@ -331,15 +317,19 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
         }
       }
       if (need) {
-        l_run *= fast_exp2(m_run - m_new);
+        const float f = fast_exp2(m_run - m_new);
+        l_run *= f;
+        l_mma *= f;
         m_run = m_new;
       }
       const float neg_m = -m_run;
-      float s0 = 0.f, s1 = 0.f;
+      float e0 = 0.f, e1 = 0.f, q0 = 0.f, q1 = 0.f;
       // Exponentiate 32 columns at a time and store them as 16 packed bf16
-      // pairs right away, so at most 16 P words are live at once. The row sum
-      // adds the bf16-rounded values the PV MMA consumes, so numerator and
-      // denominator see the same weights (a one-hot row returns V exactly).
+      // pairs right away, so at most 16 P words are live at once. Two row sums
+      // are kept. The exact one (unrounded p) gives lse. The other adds the
+      // bf16-rounded p that the PV MMA consumes, and O is divided by it, so
+      // O's weights sum to one as they do in the definition (a one-hot row
+      // returns V exactly).
       auto emit = [&](const uint32_t (&r)[32], uint32_t col) {
         uint32_t pw[16];
 #pragma unroll
@@ -348,7 +338,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
           const float x1 = fast_exp2(fmaf(u2f(r[2 * e + 1]), scale_log2, neg_m));
           const uint32_t pk = pack_bf16x2(x0, x1);
           const float rounded = u2f(pk << 16) + u2f(pk & 0xFFFF0000u);
-          if (e & 1) s1 += rounded; else s0 += rounded;
+          if (e & 1) { e1 += x0 + x1; q1 += rounded; } else { e0 += x0 + x1; q0 += rounded; }
           pw[e] = pk;
         }
         tmem_st16(t_p + col, pw);
@@ -357,7 +347,8 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
       emit(r1, 16);
       emit(r2, 32);
       emit(r3, 48);
-      l_run += s0 + s1;
+      l_run += e0 + e1;
+      l_mma += q0 + q1;
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(&p_full[t]);
@@ -366,7 +357,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
     if (ok) ok = mbar_wait(&o_full[t], 0, abort_flag, kSiteOFull);
     if (ok) {
       tc_fence_after();
-      const float inv_l = 1.0f / l_run;
+      const float inv_l = 1.0f / l_mma;
       __nv_bfloat16* orow = out + (static_cast<size_t>(bh) * N + row) * D;
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {

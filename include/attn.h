@@ -112,6 +112,20 @@ attn_status attn_check_status(attn_stream_t stream);
  * owns the string. It stays valid until the next call on the same thread. */
 const char* attn_get_last_error(void);
 
+/*
+ * Opt-in per-kernel timing (tracing). While enabled, each kernel launch is
+ * bracketed by two CUDA events recorded on its stream. The events come from
+ * a pool that the library creates on first use. attn_profile_read() waits for
+ * the recorded events and returns, for kernel index `kernel` (0 fwd_kernel,
+ * 1 bwd_pre_kernel, 2 bwd_dkdv_kernel, 3 bwd_dq_kernel), its name, the number
+ * of launches timed and their summed duration in milliseconds since the last
+ * reset. An out-of-range index returns ATTN_ERR_ARG. Off by default. When it
+ * is off, calls record nothing.
+ */
+void attn_profile_enable(int on);
+void attn_profile_reset(void);
+attn_status attn_profile_read(int kernel, const char** name, int* launches, double* total_ms);
+
 /* ABI version of this header: major * 100 + minor. */
 int attn_abi_version(void);
 
