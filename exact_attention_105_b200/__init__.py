@@ -29,6 +29,8 @@ SIGNATURES = {
     "attn_bwd": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _SZ,
                       _I, _I, _I, _I, _I, _F, _I, _P]),
     "attn_bwd_workspace_size": (_SZ, [_I, _I, _I, _I]),
+    "attn_bwd_noalloc": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P,
+                              _I, _I, _I, _I, _I, _F, _I, _P]),
     "attn_check_status": (_I, [_P]),
     "attn_get_last_error": (ctypes.c_char_p, []),
     "attn_abi_version": (_I, []),
@@ -154,6 +156,27 @@ def attn_bwd(q, k, v, o, lse, dO, dq=None, dk=None, dv=None, workspace=None, sca
                         _dev_ptr(dk, "dk"), _dev_ptr(dv, "dv"), _dev_ptr(workspace, "workspace"),
                         workspace.numel() * workspace.element_size(),
                         B, Hq, Hkv, N, d, scale, int(bool(causal)), _stream_handle(stream)))
+    return dq, dk, dv
+
+
+NOALLOC_SCRATCH_BYTES = 8 << 20
+
+
+def attn_bwd_noalloc(q, k, v, o, lse, dO, dq, dk, dv, scale=None, causal=False, stream=None):
+    """attn_bwd without a workspace, for callers that must not allocate device
+    memory when the backward runs. The scratch is a fixed 8 MiB device array
+    inside the library (shapes with B * Hq * ceil128(N) > 1048576 are rejected),
+    and the output tensors must be passed in. Calls that
+    overlap on the GPU share that array and race. Returns (dq, dk, dv)."""
+    B, Hq, N, d = q.shape
+    Hkv = k.shape[1]
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    lib = load_library()
+    _check(lib.attn_bwd_noalloc(_dev_ptr(q, "q"), _dev_ptr(k, "k"), _dev_ptr(v, "v"),
+                                _dev_ptr(o, "o"), _dev_ptr(lse, "lse"), _dev_ptr(dO, "dO"),
+                                _dev_ptr(dq, "dq"), _dev_ptr(dk, "dk"), _dev_ptr(dv, "dv"),
+                                B, Hq, Hkv, N, d, scale, int(bool(causal)),
+                                _stream_handle(stream)))
     return dq, dk, dv
 
 

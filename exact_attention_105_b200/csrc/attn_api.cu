@@ -287,6 +287,40 @@ attn_status launch_bwd(const BwdArgs& a, cudaStream_t stream) {
   return ATTN_OK;
 }
 
+// ---------------------------------------------------------------- static scratch
+// Backing store for attn_bwd_noalloc: the backward's lse*log2(e) and
+// rowsum(dO*O) rows live in this fixed device array instead of a
+// caller-provided workspace. Every device that loads the library holds these
+// 8 MiB until the process exits. Host code must not hand the symbol itself to
+// a kernel (on the host it names a stand-in, not device memory). Its device
+// address is looked up once per device with cudaGetSymbolAddress.
+constexpr size_t kStaticScratchBytes = size_t(8) << 20;
+static __device__ __align__(256) float g_bwd_scratch[kStaticScratchBytes / sizeof(float)];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_scratch_mu;
+void* g_scratch_addr[kMaxDevices] = {};
+
+// Device address of g_bwd_scratch on the current device. The first call on
+// each device resolves it (with that device current) and caches it.
+attn_status static_scratch_ptr(void** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= kMaxDevices) return fail(ATTN_ERR_CUDA, "device index %d unsupported", dev);
+  std::lock_guard<std::mutex> g(g_scratch_mu);
+  if (g_scratch_addr[dev] == nullptr) {
+    void* ptr = nullptr;
+    e = cudaGetSymbolAddress(&ptr, g_bwd_scratch);
+    if (e != cudaSuccess || ptr == nullptr)
+      return cuda_fail(e != cudaSuccess ? e : cudaErrorInvalidSymbol,
+                       "cudaGetSymbolAddress(static backward scratch)");
+    g_scratch_addr[dev] = ptr;
+  }
+  *out = g_scratch_addr[dev];
+  return ATTN_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -362,6 +396,49 @@ attn_status attn_bwd(const void* q, const void* k, const void* v, const void* o,
   if ((st = make_map(&mv, v, d, N, B * Hkv)) != ATTN_OK) return st;
   if ((st = make_map(&mdo, dO, d, N, B * Hq)) != ATTN_OK) return st;
   float* L = static_cast<float*>(workspace);
+  float* Dv = L + static_cast<size_t>(B) * Hq * attn::pad128(N);
+  BwdArgs a{mq, mk, mv, mdo, o, lse, dO, dq, dk, dv, L, Dv, B, Hq, Hkv, N, scale};
+  if (d == 64) return causal ? launch_bwd<64, true>(a, stream) : launch_bwd<64, false>(a, stream);
+  return causal ? launch_bwd<128, true>(a, stream) : launch_bwd<128, false>(a, stream);
+}
+
+attn_status attn_bwd_noalloc(const void* q, const void* k, const void* v, const void* o,
+                             const float* lse, const void* dO, void* dq, void* dk, void* dv,
+                             int B, int Hq, int Hkv, int N, int d, float scale, int causal,
+                             attn_stream_t stream_) {
+  g_last_error[0] = '\0';
+  bool empty = false;
+  attn_status st = check_shape(B, Hq, Hkv, N, d, scale, &empty);
+  if (st != ATTN_OK) return st;
+  if (causal != 0 && causal != 1) return fail(ATTN_ERR_ARG, "causal must be 0 or 1");
+  if (empty) return ATTN_OK;
+  const void* ptrs[9] = {q, k, v, o, lse, dO, dq, dk, dv};
+  const char* names[9] = {"q", "k", "v", "o", "lse", "dO", "dq", "dk", "dv"};
+  for (int i = 0; i < 9; ++i) {
+    if (ptrs[i] == nullptr) return fail(ATTN_ERR_ARG, "%s is null", names[i]);
+    if (!aligned16(ptrs[i])) return fail(ATTN_ERR_ARG, "%s is not 16-byte aligned", names[i]);
+  }
+  const size_t need = attn_bwd_workspace_size(B, Hq, N, d);
+  if (need > kStaticScratchBytes)
+    return fail(ATTN_ERR_ARG,
+                "attn_bwd_noalloc: this shape needs %zu bytes of scratch, but the static area "
+                "holds %zu (B*Hq*ceil128(N) must be <= %zu); use attn_bwd with a workspace",
+                need, kStaticScratchBytes, kStaticScratchBytes / (2 * sizeof(float)));
+  st = ensure_init();
+  if (st != ATTN_OK) return st;
+  if ((st = check_ptrs(ptrs, names, 9)) != ATTN_OK) return st;
+  void* scratch = nullptr;
+  if ((st = static_scratch_ptr(&scratch)) != ATTN_OK) return st;
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+  CUtensorMap mq, mk, mv, mdo;
+  if ((st = make_map(&mq, q, d, N, B * Hq)) != ATTN_OK) return st;
+  if ((st = make_map(&mk, k, d, N, B * Hkv)) != ATTN_OK) return st;
+  if ((st = make_map(&mv, v, d, N, B * Hkv)) != ATTN_OK) return st;
+  if ((st = make_map(&mdo, dO, d, N, B * Hq)) != ATTN_OK) return st;
+  // The preprocess kernel writes every scratch row the other two kernels read,
+  // so nothing left over from an earlier call is ever used and no clearing
+  // is needed.
+  float* L = static_cast<float*>(scratch);
   float* Dv = L + static_cast<size_t>(B) * Hq * attn::pad128(N);
   BwdArgs a{mq, mk, mv, mdo, o, lse, dO, dq, dk, dv, L, Dv, B, Hq, Hkv, N, scale};
   if (d == 64) return causal ? launch_bwd<64, true>(a, stream) : launch_bwd<64, false>(a, stream);

@@ -102,6 +102,38 @@ attn_status attn_bwd(const void* q, const void* k, const void* v, const void* o,
 size_t attn_bwd_workspace_size(int B, int Hq, int N, int d);
 
 /*
+ * attn_bwd_noalloc: attn_bwd for callers that cannot allocate device memory.
+ * Some callers cannot call cudaMalloc, or any allocator, at the point where
+ * they run the backward pass. Examples: plugins whose execute step must not
+ * allocate, code running inside an allocator or memory-pool callback, and
+ * processes that place all device memory at start-up under a fixed budget.
+ * Such callers cannot supply attn_bwd's workspace. This entry point takes the
+ * same tensors as attn_bwd (inputs and outputs are still caller-owned) and
+ * keeps its scratch in a fixed 8 MiB array that the library places in device
+ * memory. Every GPU that loads the library holds that array until the process
+ * exits. The pages describe no such entry point. It has no counterpart there.
+ *   - Limit: attn_bwd_workspace_size(B, Hq, N, d) must not exceed 8 MiB
+ *     (8388608 bytes), i.e. B * Hq * (N rounded up to a multiple of 128)
+ *     <= 1048576. Larger shapes return ATTN_ERR_ARG with a message, and
+ *     nothing is launched.
+ *   - It calls no cudaMalloc, cudaFree or other allocating routine. The first
+ *     call on each device looks up the array's device address
+ *     (cudaGetSymbolAddress) with that device current, and caches it. Make
+ *     that first call on a device before any stream capture.
+ *   - All calls share the one array, which keeps the last call's contents.
+ *     Each call rewrites every scratch entry it reads before reading it, so
+ *     nothing has to be cleared. Calls whose kernels overlap on the GPU (for
+ *     example on two streams without ordering between them) race on the
+ *     array and may return wrong gradients. Order such calls on one stream or
+ *     with events.
+ * Results are the same as attn_bwd's for the same inputs.
+ */
+attn_status attn_bwd_noalloc(const void* q, const void* k, const void* v, const void* o,
+                             const float* lse, const void* dO, void* dq, void* dk, void* dv,
+                             int B, int Hq, int Hkv, int N, int d, float scale, int causal,
+                             attn_stream_t stream);
+
+/*
  * Synchronises `stream`, then reads and clears the device status word.
  * Returns ATTN_ERR_TIMEOUT if a kernel gave up on a wait since the last
  * check, ATTN_ERR_CUDA on a CUDA error, and ATTN_OK otherwise.
