@@ -48,7 +48,20 @@ def parse_args():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-extra", action="store_true", help="skip the forward-only target workloads")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--mode", choices=["step", "fwd"], default="step",
+                    help="step: forward + backward (default); fwd: forward only")
+    ap.add_argument("--workload", default=None,
+                    help="workload name from workloads.py (default: the training-step config)")
     return ap.parse_args()
+
+
+def pick_workload(args):
+    if args.workload is None:
+        return WORKLOAD
+    for w in workloads.ALL:
+        if w.name == args.workload:
+            return w
+    sys.exit(f"unknown workload {args.workload!r}; choose from {[w.name for w in workloads.ALL]}")
 
 
 def load_peaks():
@@ -279,9 +292,10 @@ def run_ours(args):
         from datetime import timedelta
         dist.init_process_group("nccl", timeout=timedelta(seconds=120),
                                 device_id=torch.device("cuda", local))
-    w = WORKLOAD
-    w_rank = workloads.Workload(w.name, w.B, w.Hq, w.Hkv, w.N, w.d, w.causal, backward=True,
-                                seed=w.seed + rank)
+    w = pick_workload(args)
+    fwd_only = args.mode == "fwd"
+    w_rank = workloads.Workload(w.name, w.B, w.Hq, w.Hkv, w.N, w.d, w.causal, q_mult=w.q_mult,
+                                backward=True, seed=w.seed + rank)
     peaks = load_peaks()
     host = workloads.make_inputs(w_rank)
     q, k, v, do = (t.cuda() for t in host)
@@ -294,7 +308,8 @@ def run_ours(args):
 
     def step():
         ea.attn_fwd(q, k, v, o, lse, scale=w.scale, causal=w.causal)
-        ea.attn_bwd(q, k, v, o, lse, do, dq, dk, dv, ws, scale=w.scale, causal=w.causal)
+        if not fwd_only:
+            ea.attn_bwd(q, k, v, o, lse, do, dq, dk, dv, ws, scale=w.scale, causal=w.causal)
 
     for _ in range(max(3, args.warmup)):
         step()
@@ -326,7 +341,7 @@ def run_ours(args):
     prof = ea.profile_read()
     launches = sum(n for n, _ in prof.values())
 
-    flops_step = w.fwd_flops() + w.bwd_flops()
+    flops_step = w.fwd_flops() + (0.0 if fwd_only else w.bwd_flops())
     value = flops_step * args.steps * world / (elapsed / 1e3) / 1e12
 
     # Roofline of the dominant kernel (largest share of the timed region).
@@ -367,12 +382,20 @@ def run_ours(args):
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
+    o_host = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
+    lse_host = torch.empty(lse.shape, dtype=lse.dtype, pin_memory=True)
     for _ in range(e2e_steps):
         for dst, src in zip((q, k, v, do), pin):
+            if fwd_only and dst is do:
+                continue
             dst.copy_(src, non_blocking=True)
         step()
-        for dst, src in zip(outs, (dq, dk, dv)):
-            dst.copy_(src, non_blocking=True)
+        if fwd_only:
+            o_host.copy_(o, non_blocking=True)
+            lse_host.copy_(lse, non_blocking=True)
+        else:
+            for dst, src in zip(outs, (dq, dk, dv)):
+                dst.copy_(src, non_blocking=True)
     e1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = e0.elapsed_time(e1)
@@ -382,11 +405,14 @@ def run_ours(args):
         e2e_ms = float(t.item())
     h2d = sum(t.numel() * t.element_size() for t in pin)
     d2h = sum(t.numel() * t.element_size() for t in outs)
+    if fwd_only:   # inputs q, k, v in; o and lse out
+        h2d -= do.numel() * do.element_size()
+        d2h = o.numel() * o.element_size() + lse.numel() * lse.element_size()
     e2e = {"value": flops_step * e2e_steps * world / (e2e_ms / 1e3) / 1e12, "unit": UNIT,
            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps}
 
     extra = None
-    if not args.no_extra and rank == 0:
+    if not args.no_extra and rank == 0 and not fwd_only:
         del pin, outs
         torch.cuda.empty_cache()
         extra = []
@@ -396,7 +422,7 @@ def run_ours(args):
             extra.append(r)
 
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and not fwd_only:
         cpu = oracle_baseline(w, host, steps=3, per_step_s=4.0)
         cpu = {k2: cpu[k2] for k2 in ("value", "unit", "cores", "kind", "sample")}
 
@@ -409,7 +435,8 @@ def run_ours(args):
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": max(3, args.warmup), "ms_per_step": elapsed / args.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-            "data": "synthetic (seeded iid N(0,1) -> bf16)", "config": config_dict(w, world),
+            "data": "synthetic (seeded iid N(0,1) -> bf16)",
+            "config": dict(config_dict(w, world), mode=args.mode),
             "frac_of_peak": value / peaks["bf16_tflops"],
             "roofline": roofline, "kernels": kernels, "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": launches, "clocks": clocks, "fwd_targets": extra,

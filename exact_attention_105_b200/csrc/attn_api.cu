@@ -12,6 +12,7 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <algorithm>
 #include <mutex>
 #include <vector>
 
@@ -96,6 +97,7 @@ using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t
                                    CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
 EncodeTiledFn g_encode = nullptr;
+int g_num_sms = 148;
 attn_status g_init_status = ATTN_OK;
 char g_init_msg[256] = "";
 std::once_flag g_init_once;
@@ -126,6 +128,7 @@ void init_once() {
     return;
   }
   g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+  g_num_sms = prop.multiProcessorCount > 0 ? prop.multiProcessorCount : 148;
 }
 
 attn_status ensure_init() {
@@ -215,7 +218,9 @@ attn_status launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUten
   if (launch_regs != attn::kFwdRegsLaunch)
     return fail(ATTN_ERR_CUDA, "fwd kernel built with %d registers/thread, expected %d",
                 launch_regs, attn::kFwdRegsLaunch);
-  dim3 grid(B * Hq, (N + 255) / 256);
+  const long long blocks = static_cast<long long>(B) * Hq * ((N + 255) / 256);
+  if (blocks > 0x7FFFFFFFLL) return fail(ATTN_ERR_ARG, "problem too large for one launch");
+  dim3 grid(static_cast<unsigned>(blocks));
   const float scale_log2 = scale * 1.4426950408889634f;
   ProfScope ps(kProfFwd, stream);
   kern<<<grid, Cfg::kThreads, Cfg::kSmemAlloc, stream>>>(
@@ -255,6 +260,9 @@ attn_status launch_bwd(const BwdArgs& a, cudaStream_t stream) {
   const float scale_log2 = a.scale * kLog2e;
 
   const long long rows = static_cast<long long>(a.B) * a.Hq * Npad;
+  const long long g1 = static_cast<long long>(nblk) * a.B * a.Hkv;
+  const long long g2 = static_cast<long long>(nblk) * a.B * a.Hq;
+  if (rows / 32 > 0x7FFFFFFFLL) return fail(ATTN_ERR_ARG, "problem too large for one launch");
   ProfScope p0(kProfBwdPre, stream);
   bwd_pre_kernel<D><<<static_cast<unsigned>(rows / 32), 256, 0, stream>>>(
       static_cast<const __nv_bfloat16*>(a.o), static_cast<const __nv_bfloat16*>(a.dO), a.lse,
@@ -273,13 +281,13 @@ attn_status launch_bwd(const BwdArgs& a, cudaStream_t stream) {
     return cuda_fail(e, "cudaFuncSetAttribute(dq)");
 
   ProfScope p1(kProfBwdDkdv, stream);
-  k1<<<dim3(a.B * a.Hkv, nblk), DkdvCfg<D>::kThreads, DkdvCfg<D>::kSmemAlloc, stream>>>(
+  k1<<<dim3(static_cast<unsigned>(g1)), DkdvCfg<D>::kThreads, DkdvCfg<D>::kSmemAlloc, stream>>>(
       a.mq, a.mk, a.mv, a.mdo, a.L, a.Dv, static_cast<__nv_bfloat16*>(a.dk),
       static_cast<__nv_bfloat16*>(a.dv), a.Hq, group, a.N, Npad, scale_log2, a.scale);
   p1.end();
   if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "bwd dK/dV launch");
   ProfScope p2(kProfBwdDq, stream);
-  k2<<<dim3(a.B * a.Hq, nblk), DqCfg<D>::kThreads, DqCfg<D>::kSmemAlloc, stream>>>(
+  k2<<<dim3(static_cast<unsigned>(g2)), DqCfg<D>::kThreads, DqCfg<D>::kSmemAlloc, stream>>>(
       a.mq, a.mk, a.mv, a.mdo, a.L, a.Dv, static_cast<__nv_bfloat16*>(a.dq), a.Hq, group, a.N,
       Npad, scale_log2, a.scale);
   p2.end();

@@ -11,9 +11,10 @@
 // D = rowsum(dO * O) equals rowsum(P * dP) because O = P V.
 //
 // Three kernels, all deterministic (no atomics):
-//   bwd_pre_kernel   D and lse * log2(e), per query row, into the workspace,
+//   bwd_pre_kernel   -D and -lse * log2(e), per query row, into the workspace
+//                    (negated so P and dS are one paired fma/add each),
 //                    padded to a multiple of 128 rows per head. Padding rows
-//                    get lse = +inf, so every P that involves them is 0.
+//                    get -lse = -inf, so every P that involves them is 0.
 //   bwd_dkdv_kernel  one CTA per (batch, KV head, 128-key block). K_j and V_j
 //                    stay in shared memory. It loops over the 128-query blocks
 //                    of every query head in the GQA group (from the diagonal
@@ -22,9 +23,14 @@
 //   bwd_dq_kernel    one CTA per (batch, query head, 128-query block). Q_i and
 //                    dO_i stay resident while K_j/V_j stream through a ring. Per
 //                    block it computes S, dP, P, dS and accumulates dQ in TMEM.
-// Warp roles in both main kernels (256 threads): warps 0-3 compute (thread r
-// owns TMEM lane r), warp 4 TMA producer, warp 5 TMEM allocator and MMA
-// issuer, warps 6-7 idle.
+// Warp roles in both main kernels (384 threads): warps 0-7 are two compute
+// warpgroups, warp 8 is the TMA producer, warp 9 allocates TMEM and issues
+// the MMAs, and warps 10-11 idle. Thread r of a compute warpgroup owns TMEM
+// lane r. Warpgroup h owns columns [64h, 64h+64) of the step's 128x128 S and
+// dP tiles. It writes its bf16 P/dS pairs back into the first 32 of its own
+// 64 columns, so neither group overwrites columns the other has yet to read.
+// The MMA that consumes them reads K-step kk (16 columns) from TMEM column
+// 64*(kk/4) + 8*(kk%4) of the tile.
 #pragma once
 
 #include "sm100.cuh"
@@ -69,8 +75,8 @@ bwd_pre_kernel(const __nv_bfloat16* __restrict__ o, const __nv_bfloat16* __restr
   acc += __shfl_xor_sync(0xffffffffu, acc, 2);
   acc += __shfl_xor_sync(0xffffffffu, acc, 1);
   if (sub == 0) {
-    L[row] = (n < N) ? lse[static_cast<size_t>(bh) * N + n] * kLog2e : INFINITY;
-    Dv[row] = (n < N) ? acc : 0.f;
+    L[row] = (n < N) ? -lse[static_cast<size_t>(bh) * N + n] * kLog2e : -INFINITY;
+    Dv[row] = (n < N) ? -acc : 0.f;
   }
 }
 
@@ -93,27 +99,30 @@ __device__ __forceinline__ void tmem_ld128(uint32_t taddr, uint32_t (&r0)[32], u
   reg_fence(r3);
 }
 
-// dS = P * (dP - Dcol) for 32 columns, P given as 16 packed bf16 pairs;
-// writes 16 packed bf16 pairs of dS. `dsub(e)` gives the D value of column e.
-template <typename DSub>
-__device__ __forceinline__ void ds_block(const uint32_t* pw, const uint32_t (&dp)[32],
-                                         uint32_t* out, DSub dsub) {
+// dS = P * (dP - D) for 32 columns, P in fp32, given -D per column pair as
+// float2 through `nd(e)` (e even); writes 16 packed bf16 pairs of dS.
+template <typename NegD>
+__device__ __forceinline__ void ds_block(const float* pf, const uint32_t (&dp)[32],
+                                         uint32_t* out, NegD nd) {
 #pragma unroll
   for (int e = 0; e < 16; ++e) {
-    const float p0 = u2f(pw[e] << 16), p1 = u2f(pw[e] & 0xFFFF0000u);
-    const float a = p0 * (u2f(dp[2 * e]) - dsub(2 * e));
-    const float b = p1 * (u2f(dp[2 * e + 1]) - dsub(2 * e + 1));
-    out[e] = pack_bf16x2(a, b);
+    const float2 d = fadd2(make_float2(u2f(dp[2 * e]), u2f(dp[2 * e + 1])), nd(2 * e));
+    const float2 v = fmul2(make_float2(pf[2 * e], pf[2 * e + 1]), d);
+    out[e] = pack_bf16x2(v.x, v.y);
   }
 }
 
+// TMEM column offset of K-step kk (16 bf16 columns) of a P / dS tile whose
+// two 64-column halves were packed into the first 32 columns of each half.
+__device__ __forceinline__ uint32_t split_col(int kk) { return 64 * (kk >> 2) + 8 * (kk & 3); }
+
 // Epilogue helper: one 128 x D fp32 accumulator row (this thread's lane) ->
 // bf16 * mul, stored to `dst` when `valid`.
-template <int D>
+template <int D, int C0 = 0, int C1 = D / 32>
 __device__ __forceinline__ void store_acc_row(uint32_t t_acc, __nv_bfloat16* dst, float mul,
                                               bool valid) {
 #pragma unroll
-  for (int c = 0; c < D / 32; ++c) {
+  for (int c = C0; c < C1; ++c) {
     uint32_t a[32];
     tmem_ld32(t_acc + c * 32, a);
     tmem_ld_wait(a);
@@ -145,11 +154,11 @@ struct DkdvCfg {
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
   static constexpr int kBytes = kMiscOff + 16;
   static constexpr int kSmemAlloc = kBytes + 1024;
-  static constexpr int kThreads = 256;
+  static constexpr int kThreads = 384;
 };
 
 template <int D, bool CAUSAL>
-__global__ void __launch_bounds__(256, 1)
+__global__ void __launch_bounds__(384, 1)
 bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
                 const float* __restrict__ Lws, const float* __restrict__ Dws,
@@ -175,11 +184,14 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 
   const int warp = warp_id(), lane = lane_id();
   const int Hkv = Hq / group;
-  const int bh_kv = blockIdx.x;
+  // 1-D grid, KV block fastest, then (batch, KV head): CTAs resident
+  // together mostly share one head's Q/dO in L2. Low j has the most causal
+  // work and launches first within its head.
+  const int nq = (N + 127) >> 7;
+  const int bh_kv = blockIdx.x / nq;
   const int b = bh_kv / Hkv;
   const int hkv = bh_kv - b * Hkv;
-  const int j = blockIdx.y;                   // KV block: low j has the most causal work
-  const int nq = (N + 127) >> 7;
+  const int j = blockIdx.x - bh_kv * nq;
   const int i_start = CAUSAL ? j : 0;
   const int per_head = nq - i_start;
   const int n_steps = group * per_head;       // >= 1
@@ -192,14 +204,14 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     }
     mbar_init(s_full, 1);
     mbar_init(dp_full, 1);
-    mbar_init(p_full, 128);
-    mbar_init(ds_full, 128);
+    mbar_init(p_full, 256);
+    mbar_init(ds_full, 256);
     mbar_init(acc_done, 1);
     mbar_init(mma_done, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 5) {
+  if (warp == 9) {
     tmem_alloc(tmem_slot, 512);
     tmem_relinquish();
   }
@@ -214,7 +226,7 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     bh_q = b * Hq + hkv * group + g;
   };
 
-  if (warp == 4) {
+  if (warp == 8) {
     if (lane == 0) {
       // -------------------------------------------------------- producer
       tma_prefetch_desc(&tm_q);
@@ -249,7 +261,7 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       const int first = issued > NS ? issued - NS : 0;
       for (int s = first; s < issued; ++s) mbar_wait_drain(&ld_full[s % NS], (s / NS) & 1);
     }
-  } else if (warp == 5) {
+  } else if (warp == 9) {
     if (lane == 0) {
       // -------------------------------------------------------- MMA issuer
       constexpr uint32_t kIdescSS = idesc_bf16_f32(128, 128, 0, 0);
@@ -264,11 +276,11 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                  kk > 0 ? 1u : 0u);
         }
       };
-      // acc(tmem) += A(tmem, 128 x 128 bf16) * B(smem tile, MN-major), K = 128
+      // acc(tmem) += A(tmem, 128 x 128 bf16, split layout) * B(smem tile, MN-major), K = 128
       auto mma_acc = [&](uint32_t acc, uint32_t a_tmem, uint32_t b, bool accumulate) {
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-          mma_ts(acc, a_tmem + kk * 8, sdesc_sw128(b + kk * 2048, 16384, 1024), kIdescAcc,
+          mma_ts(acc, a_tmem + split_col(kk), sdesc_sw128(b + kk * 2048, 16384, 1024), kIdescAcc,
                  (accumulate || kk > 0) ? 1u : 0u);
       };
       bool ok = mbar_wait(kv_full, 0, abort_flag, kSiteBKV) &&
@@ -284,7 +296,7 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         const uint32_t sa = stage_addr(s);
         if (!mbar_wait(p_full, s & 1, abort_flag, kSiteBP)) { ok = false; break; }
         tc_fence_after();
-        mma_acc(tmem + 256, tmem + 64, sa + C::kTile, s > 0);                     // dV += P^T dO
+        mma_acc(tmem + 256, tmem + 0, sa + C::kTile, s > 0);                      // dV += P^T dO
         const bool more = s + 1 < n_steps;
         if (more) {
           if (!mbar_wait(&ld_full[(s + 1) % NS], ((s + 1) / NS) & 1, abort_flag, kSiteBLoadFull)) {
@@ -297,7 +309,7 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         }
         if (!mbar_wait(ds_full, s & 1, abort_flag, kSiteBDS)) { ok = false; break; }
         tc_fence_after();
-        mma_acc(tmem + 384, tmem + 192, sa, s > 0);                               // dK += dS^T Q
+        mma_acc(tmem + 384, tmem + 128, sa, s > 0);                               // dK += dS^T Q
         tc_commit(&ld_empty[s % NS]);
         if (more) {
           mma_tile_kk(tmem + 128, sbase + C::kVOff, stage_addr(s + 1) + C::kTile); // dP^T(s+1)
@@ -309,19 +321,23 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       mbar_wait_drain(mma_done, 0);
     }
     __syncwarp();
-  } else if (warp < 4) {
+  } else if (warp < 8) {
     // ---------------------------------------------------------- compute
-    const int t = warp * 32 + lane;                   // key row within the block
+    const int h = warp >> 2;                          // column half of the step tile
+    const int quad = warp & 3;
+    const int t = quad * 32 + lane;                   // key row within the block
     const int key = j * 128 + t;
-    const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
-    const uint32_t t_s = tmem + lane_base;            // S^T, P^T at +64
-    const uint32_t t_dp = tmem + lane_base + 128;     // dP^T, dS^T at +64
+    const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
+    const uint32_t t_s = tmem + lane_base + 64 * h;          // S^T half; P^T into +0..32
+    const uint32_t t_dp = tmem + lane_base + 128 + 64 * h;   // dP^T half; dS^T into +0..32
+    const int c_base = 64 * h;
     bool ok = true;
     for (int s = 0; ok && s < n_steps; ++s) {
       int i, bh_q;
       step_head(s, i, bh_q);
       const int st = s % NS;
-      const float* Ls = reinterpret_cast<const float*>(smem + C::kStageOff + st * C::kStageBytes + 2 * C::kTile);
+      const float* Ls = reinterpret_cast<const float*>(smem + C::kStageOff + st * C::kStageBytes +
+                                                       2 * C::kTile) + c_base;
       const float* Ds = Ls + 128;
       if (!mbar_wait(&ld_full[st], (s / NS) & 1, abort_flag, kSiteBLoadFull) ||
           !mbar_wait(s_full, s & 1, abort_flag, kSiteBS)) {
@@ -329,60 +345,54 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         break;
       }
       tc_fence_after();
-      uint32_t r0[32], r1[32], r2[32], r3[32];
-      tmem_ld128(t_s, r0, r1, r2, r3);
+      uint32_t r0[32], r1[32];
+      tmem_ld32(t_s, r0);
+      tmem_ld32(t_s + 32, r1);
+      tmem_ld_wait(r0);
+      reg_fence(r1);
       const bool diag = CAUSAL && (i == j);           // key t sees query c only if c >= t
-      uint32_t pw[64];
+      const float2 sc2 = make_float2(scale_log2, scale_log2);
+      float pf[64];                                   // P in fp32 (for dS)
+      uint32_t pw[32];                                // P as bf16 pairs (for the dV MMA)
       auto p_block = [&](const uint32_t (&r)[32], int c0) {
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
-          const int c = c0 + 2 * e;
-          float p0 = fast_exp2(fmaf(u2f(r[2 * e]), scale_log2, -Ls[c]));
-          float p1 = fast_exp2(fmaf(u2f(r[2 * e + 1]), scale_log2, -Ls[c + 1]));
+          const int c = c_base + c0 + 2 * e;
+          const float2 nl = *reinterpret_cast<const float2*>(&Ls[c0 + 2 * e]);
+          const float2 x = ffma2(make_float2(u2f(r[2 * e]), u2f(r[2 * e + 1])), sc2, nl);
+          float p0 = fast_exp2(x.x);
+          float p1 = fast_exp2(x.y);
           if (diag) {
             if (c < t) p0 = 0.f;
             if (c + 1 < t) p1 = 0.f;
           }
+          pf[c0 + 2 * e] = p0;
+          pf[c0 + 2 * e + 1] = p1;
           pw[c0 / 2 + e] = pack_bf16x2(p0, p1);
         }
       };
       p_block(r0, 0);
       p_block(r1, 32);
-      p_block(r2, 64);
-      p_block(r3, 96);
-#pragma unroll
-      for (int c = 0; c < 4; ++c) tmem_st16(t_s + 64 + 16 * c, &pw[16 * c]);
+      tmem_st16(t_s, &pw[0]);
+      tmem_st16(t_s + 16, &pw[16]);
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(p_full);
 
       if (!mbar_wait(dp_full, s & 1, abort_flag, kSiteBDP)) { ok = false; break; }
       tc_fence_after();
-      // dS^T goes to dP^T columns [64,128): read those dP^T columns first.
-      uint32_t d2[32], d3[32];
-      tmem_ld32(t_dp + 64, d2);
-      tmem_ld32(t_dp + 96, d3);
-      tmem_ld_wait(d2);
-      reg_fence(d3);
+      uint32_t d0[32], d1[32];
+      tmem_ld32(t_dp, d0);
+      tmem_ld32(t_dp + 32, d1);
+      tmem_ld_wait(d0);
+      reg_fence(d1);
       uint32_t ds[16];
-      {
-        uint32_t d0[32];
-        tmem_ld32(t_dp + 0, d0);
-        tmem_ld_wait(d0);
-        ds_block(&pw[0], d0, ds, [&](int e) { return Ds[e]; });
-        tmem_st16(t_dp + 64, ds);
-      }
-      {
-        uint32_t d1[32];
-        tmem_ld32(t_dp + 32, d1);
-        tmem_ld_wait(d1);
-        ds_block(&pw[16], d1, ds, [&](int e) { return Ds[32 + e]; });
-        tmem_st16(t_dp + 80, ds);
-      }
-      ds_block(&pw[32], d2, ds, [&](int e) { return Ds[64 + e]; });
-      tmem_st16(t_dp + 96, ds);
-      ds_block(&pw[48], d3, ds, [&](int e) { return Ds[96 + e]; });
-      tmem_st16(t_dp + 112, ds);
+      ds_block(&pf[0], d0, ds,
+               [&](int e) { return *reinterpret_cast<const float2*>(&Ds[e]); });
+      tmem_st16(t_dp, ds);
+      ds_block(&pf[32], d1, ds,
+               [&](int e) { return *reinterpret_cast<const float2*>(&Ds[32 + e]); });
+      tmem_st16(t_dp + 16, ds);
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(ds_full);
@@ -392,14 +402,16 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       tc_fence_after();
       const bool valid = key < N;
       const size_t row_off = (static_cast<size_t>(bh_kv) * N + (valid ? key : 0)) * D;
-      store_acc_row<D>(tmem + lane_base + 256, dv + row_off, 1.0f, valid);
-      store_acc_row<D>(tmem + lane_base + 384, dk + row_off, scale, valid);
+      if (h == 0)
+        store_acc_row<D>(tmem + lane_base + 256, dv + row_off, 1.0f, valid);
+      else
+        store_acc_row<D>(tmem + lane_base + 384, dk + row_off, scale, valid);
     }
   }
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == 9) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
@@ -419,11 +431,11 @@ struct DqCfg {
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
   static constexpr int kBytes = kMiscOff + 16;
   static constexpr int kSmemAlloc = kBytes + 1024;
-  static constexpr int kThreads = 256;
+  static constexpr int kThreads = 384;
 };
 
 template <int D, bool CAUSAL>
-__global__ void __launch_bounds__(256, 1)
+__global__ void __launch_bounds__(384, 1)
 bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
               const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
               const float* __restrict__ Lws, const float* __restrict__ Dws,
@@ -448,12 +460,14 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kMiscOff + 4);
 
   const int warp = warp_id(), lane = lane_id();
-  const int bh = blockIdx.x;
+  // 1-D grid, query block fastest (heaviest causal block first), then
+  // (batch, query head): CTAs resident together mostly share one head's K/V.
+  const int nkv = (N + 127) >> 7;
+  const int bh = blockIdx.x / nkv;
   const int b = bh / Hq;
   const int hq = bh - b * Hq;
   const int bh_kv = b * (Hq / group) + hq / group;
-  const int nkv = (N + 127) >> 7;
-  const int i = gridDim.y - 1 - blockIdx.y;  // heaviest causal query blocks first
+  const int i = nkv - 1 - (blockIdx.x - bh * nkv);
   const int n = CAUSAL ? min(i + 1, nkv) : nkv;
 
   if (threadIdx.x == 0) {
@@ -463,15 +477,15 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
       mbar_init(&kv_empty[s], 1);
     }
     mbar_init(s_full, 1);
-    mbar_init(s_free, 128);
+    mbar_init(s_free, 256);
     mbar_init(dp_full, 1);
-    mbar_init(ds_full, 128);
+    mbar_init(ds_full, 256);
     mbar_init(acc_done, 1);
     mbar_init(mma_done, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 5) {
+  if (warp == 9) {
     tmem_alloc(tmem_slot, 512);
     tmem_relinquish();
   }
@@ -480,7 +494,7 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 4) {
+  if (warp == 8) {
     if (lane == 0) {
       // -------------------------------------------------------- producer
       tma_prefetch_desc(&tm_q);
@@ -514,7 +528,7 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
       const uint32_t first = issued > (uint32_t)NS ? issued - NS : 0u;
       for (uint32_t x = first; x < issued; ++x) mbar_wait_drain(&kv_full[x % NS], (x / NS) & 1u);
     }
-  } else if (warp == 5) {
+  } else if (warp == 9) {
     if (lane == 0) {
       // -------------------------------------------------------- MMA issuer
       constexpr uint32_t kIdescSS = idesc_bf16_f32(128, 128, 0, 0);
@@ -560,7 +574,7 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         const uint32_t kb = slot(ik);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)                           // dQ += dS K_j
-          mma_ts(tmem + 256, tmem + 192 + kk * 8, sdesc_sw128(kb + kk * 2048, 16384, 1024),
+          mma_ts(tmem + 256, tmem + 128 + split_col(kk), sdesc_sw128(kb + kk * 2048, 16384, 1024),
                  kIdescAcc, (jj > 0 || kk > 0) ? 1u : 0u);
         tc_commit(&kv_empty[ik % NS]);
         tc_commit(&kv_empty[iv % NS]);
@@ -576,76 +590,71 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
       mbar_wait_drain(mma_done, 0);
     }
     __syncwarp();
-  } else if (warp < 4) {
+  } else if (warp < 8) {
     // ---------------------------------------------------------- compute
-    const int t = warp * 32 + lane;                  // query row within the block
+    const int h = warp >> 2;                         // column half of the step tile
+    const int quad = warp & 3;
+    const int t = quad * 32 + lane;                  // query row within the block
     const int row = i * 128 + t;
-    const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
-    const uint32_t t_s = tmem + lane_base;
-    const uint32_t t_dp = tmem + lane_base + 128;
+    const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
+    const uint32_t t_s = tmem + lane_base + 64 * h;
+    const uint32_t t_dp = tmem + lane_base + 128 + 64 * h;   // dP half; dS into +0..32
+    const int c_base = 64 * h;
     const size_t ws = static_cast<size_t>(bh) * Npad + row;   // row < Npad always
-    const float Lr = Lws[ws];                                 // +inf on padding rows
-    const float Dr = Dws[ws];
+    const float nLr = Lws[ws];                                // -lse*log2e; -inf on padding rows
+    const float nDr = Dws[ws];                                // -rowsum(dO*O)
     bool ok = true;
     for (int jj = 0; ok && jj < n; ++jj) {
       if (!mbar_wait(s_full, jj & 1, abort_flag, kSiteBS)) { ok = false; break; }
       tc_fence_after();
-      uint32_t r0[32], r1[32], r2[32], r3[32];
-      tmem_ld128(t_s, r0, r1, r2, r3);
+      uint32_t r0[32], r1[32];
+      tmem_ld32(t_s, r0);
+      tmem_ld32(t_s + 32, r1);
+      tmem_ld_wait(r0);
+      reg_fence(r1);
       tc_fence_before();
       mbar_arrive(s_free);
       const bool diag = CAUSAL && (jj == i);          // query t sees key c only if c <= t
       // Keys past N (zero rows from the TMA fill) get P = 0 explicitly, so an
       // extreme lse can never turn 0 * exp2(-lse) into a NaN.
       const int klim = (jj == nkv - 1) ? N - jj * 128 : 128;
-      uint32_t pw[64];
+      const float2 sc2 = make_float2(scale_log2, scale_log2);
+      const float2 nl2 = make_float2(nLr, nLr);
+      float pf[64];                                   // P in fp32
       auto p_block = [&](const uint32_t (&r)[32], int c0) {
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
-          const int c = c0 + 2 * e;
-          float p0 = fast_exp2(fmaf(u2f(r[2 * e]), scale_log2, -Lr));
-          float p1 = fast_exp2(fmaf(u2f(r[2 * e + 1]), scale_log2, -Lr));
+          const int c = c_base + c0 + 2 * e;
+          const float2 x = ffma2(make_float2(u2f(r[2 * e]), u2f(r[2 * e + 1])), sc2, nl2);
+          float p0 = fast_exp2(x.x);
+          float p1 = fast_exp2(x.y);
           if (diag) {
             if (c > t) p0 = 0.f;
             if (c + 1 > t) p1 = 0.f;
           }
           if (c >= klim) p0 = 0.f;
           if (c + 1 >= klim) p1 = 0.f;
-          pw[c0 / 2 + e] = pack_bf16x2(p0, p1);
+          pf[c0 + 2 * e] = p0;
+          pf[c0 + 2 * e + 1] = p1;
         }
       };
       p_block(r0, 0);
       p_block(r1, 32);
-      p_block(r2, 64);
-      p_block(r3, 96);
 
       if (!mbar_wait(dp_full, jj & 1, abort_flag, kSiteBDP)) { ok = false; break; }
       tc_fence_after();
-      uint32_t d2[32], d3[32];
-      tmem_ld32(t_dp + 64, d2);
-      tmem_ld32(t_dp + 96, d3);
-      tmem_ld_wait(d2);
-      reg_fence(d3);
+      uint32_t d0[32], d1[32];
+      tmem_ld32(t_dp, d0);
+      tmem_ld32(t_dp + 32, d1);
+      tmem_ld_wait(d0);
+      reg_fence(d1);
       uint32_t ds[16];
-      auto dsub = [&](int) { return Dr; };
-      {
-        uint32_t d0[32];
-        tmem_ld32(t_dp + 0, d0);
-        tmem_ld_wait(d0);
-        ds_block(&pw[0], d0, ds, dsub);
-        tmem_st16(t_dp + 64, ds);
-      }
-      {
-        uint32_t d1[32];
-        tmem_ld32(t_dp + 32, d1);
-        tmem_ld_wait(d1);
-        ds_block(&pw[16], d1, ds, dsub);
-        tmem_st16(t_dp + 80, ds);
-      }
-      ds_block(&pw[32], d2, ds, dsub);
-      tmem_st16(t_dp + 96, ds);
-      ds_block(&pw[48], d3, ds, dsub);
-      tmem_st16(t_dp + 112, ds);
+      const float2 nd2 = make_float2(nDr, nDr);
+      auto nd = [&](int) { return nd2; };
+      ds_block(&pf[0], d0, ds, nd);
+      tmem_st16(t_dp, ds);
+      ds_block(&pf[32], d1, ds, nd);
+      tmem_st16(t_dp + 16, ds);
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(ds_full);
@@ -654,14 +663,17 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     if (ok) {
       tc_fence_after();
       const bool valid = row < N;
-      store_acc_row<D>(tmem + lane_base + 256, dq + (static_cast<size_t>(bh) * N + (valid ? row : 0)) * D,
-                       scale, valid);
+      __nv_bfloat16* dst = dq + (static_cast<size_t>(bh) * N + (valid ? row : 0)) * D;
+      if (h == 0)
+        store_acc_row<D, 0, D / 64>(tmem + lane_base + 256, dst, scale, valid);
+      else
+        store_acc_row<D, D / 64, D / 32>(tmem + lane_base + 256, dst, scale, valid);
     }
   }
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == 9) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }

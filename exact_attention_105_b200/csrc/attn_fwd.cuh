@@ -10,7 +10,8 @@
 //            running row max / row sum normalises it (online softmax);
 //   stage 4: O += P V accumulates in tensor memory, so the N x N matrix is
 //            never materialised;
-//   stage 5: the grid is scheduled for the B200, heavy causal blocks first.
+//   stage 5: the grid is ordered for the B200: every head's heaviest causal
+//            block first, lighter blocks after.
 //
 // CTA layout (384 threads, 12 warps):
 //   warps 0-3  softmax warpgroup for query tile 0 (rows 0..127 of the block)
@@ -97,11 +98,16 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
 
   const int warp = warp_id();
   const int lane = lane_id();
-  const int bh = blockIdx.x;                       // b * Hq + hq
+  // 1-D grid, (batch, query head) fastest, then 256-row query block from the
+  // last (heaviest when causal) to the first: every head's heaviest block is
+  // dispatched before any lighter one, which keeps the causal tail short.
+  const int nmb = (N + 255) >> 8;
+  const int BH = gridDim.x / nmb;
+  const int bh = blockIdx.x % BH;                  // b * Hq + hq
   const int b = bh / Hq;
   const int hq = bh - b * Hq;
   const int bh_kv = b * (Hq / group) + hq / group; // GQA: contiguous head groups
-  const int mb = gridDim.y - 1 - blockIdx.y;       // heaviest causal blocks launch first
+  const int mb = nmb - 1 - static_cast<int>(blockIdx.x / BH);
   const int nkv = (N + 127) >> 7;
 
   int n_t[2];
@@ -294,11 +300,11 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
       }
       float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
 #pragma unroll
-      for (int e = 0; e < 32; ++e) {
-        mx0 = fmaxf(mx0, u2f(r0[e]));
-        mx1 = fmaxf(mx1, u2f(r1[e]));
-        mx2 = fmaxf(mx2, u2f(r2[e]));
-        mx3 = fmaxf(mx3, u2f(r3[e]));
+      for (int e = 0; e < 32; e += 2) {
+        mx0 = fmax3f(mx0, u2f(r0[e]), u2f(r0[e + 1]));
+        mx1 = fmax3f(mx1, u2f(r1[e]), u2f(r1[e + 1]));
+        mx2 = fmax3f(mx2, u2f(r2[e]), u2f(r2[e + 1]));
+        mx3 = fmax3f(mx3, u2f(r3[e]), u2f(r3[e + 1]));
       }
       const float m_tile = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * scale_log2;
       const float m_new = fmaxf(m_run, m_tile);
@@ -322,23 +328,31 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
         l_mma *= f;
         m_run = m_new;
       }
-      const float neg_m = -m_run;
-      float e0 = 0.f, e1 = 0.f, q0 = 0.f, q1 = 0.f;
+      const float2 sc2 = make_float2(scale_log2, scale_log2);
+      const float2 nm2 = make_float2(-m_run, -m_run);
+      float2 ex0 = make_float2(0.f, 0.f), ex1 = make_float2(0.f, 0.f);
+      float q0 = 0.f, q1 = 0.f, q2 = 0.f, q3 = 0.f;
       // Exponentiate 32 columns at a time and store them as 16 packed bf16
       // pairs right away, so at most 16 P words are live at once. Two row sums
-      // are kept. The exact one (unrounded p) gives lse. The other adds the
-      // bf16-rounded p that the PV MMA consumes, and O is divided by it, so
-      // O's weights sum to one as they do in the definition (a one-hot row
-      // returns V exactly).
-      auto emit = [&](const uint32_t (&r)[32], uint32_t col) {
+      // are kept. The exact one (unrounded p, paired fp32 adds) gives lse. The
+      // other adds the bf16-rounded p that the PV MMA consumes, and O is divided
+      // by it, so O's weights sum to one as they do in the definition (a one-hot
+      // row returns V exactly).
+      auto emit = [&](const uint32_t (&rr)[32], uint32_t col) {
         uint32_t pw[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
-          const float x0 = fast_exp2(fmaf(u2f(r[2 * e]), scale_log2, neg_m));
-          const float x1 = fast_exp2(fmaf(u2f(r[2 * e + 1]), scale_log2, neg_m));
-          const uint32_t pk = pack_bf16x2(x0, x1);
-          const float rounded = u2f(pk << 16) + u2f(pk & 0xFFFF0000u);
-          if (e & 1) { e1 += x0 + x1; q1 += rounded; } else { e0 += x0 + x1; q0 += rounded; }
+          float2 x = ffma2(make_float2(u2f(rr[2 * e]), u2f(rr[2 * e + 1])), sc2, nm2);
+          x.x = fast_exp2(x.x);
+          x.y = fast_exp2(x.y);
+          const uint32_t pk = pack_bf16x2(x.x, x.y);
+          if (e & 1) {
+            ex1 = fadd2(ex1, x);
+            if (e & 2) q3 = add_bf16x2_to_f32(q3, pk); else q1 = add_bf16x2_to_f32(q1, pk);
+          } else {
+            ex0 = fadd2(ex0, x);
+            if (e & 2) q2 = add_bf16x2_to_f32(q2, pk); else q0 = add_bf16x2_to_f32(q0, pk);
+          }
           pw[e] = pk;
         }
         tmem_st16(t_p + col, pw);
@@ -347,8 +361,9 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
       emit(r1, 16);
       emit(r2, 32);
       emit(r3, 48);
-      l_run += e0 + e1;
-      l_mma += q0 + q1;
+      const float2 ex = fadd2(ex0, ex1);
+      l_run += ex.x + ex.y;
+      l_mma += (q0 + q1) + (q2 + q3);
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(&p_full[t]);
