@@ -617,7 +617,8 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
       const bool diag = CAUSAL && (jj == i);          // query t sees key c only if c <= t
       // Keys past N (zero rows from the TMA fill) get P = 0 explicitly, so an
       // extreme lse can never turn 0 * exp2(-lse) into a NaN.
-      const int klim = (jj == nkv - 1) ? N - jj * 128 : 128;
+      const int klim = N - jj * 128;
+      const bool ragged_tile = (jj == nkv - 1) && (N & 127) != 0;
       const float2 sc2 = make_float2(scale_log2, scale_log2);
       const float2 nl2 = make_float2(nLr, nLr);
       float pf[64];                                   // P in fp32
@@ -632,8 +633,10 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             if (c > t) p0 = 0.f;
             if (c + 1 > t) p1 = 0.f;
           }
-          if (c >= klim) p0 = 0.f;
-          if (c + 1 >= klim) p1 = 0.f;
+          if (ragged_tile) {
+            if (c >= klim) p0 = 0.f;
+            if (c + 1 >= klim) p1 = 0.f;
+          }
           pf[c0 + 2 * e] = p0;
           pf[c0 + 2 * e + 1] = p1;
         }

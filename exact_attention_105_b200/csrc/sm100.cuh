@@ -73,6 +73,22 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
+// try_wait with a suspend-time hint: the waiting thread is parked by the
+// hardware until the phase completes or about `hint_ns` pass, instead of
+// spinning and taking issue slots from the warps that do the work.
+constexpr uint32_t kWaitHintNs = 1000000;  // 1 ms per try
+__device__ __forceinline__ bool mbar_try_wait_hint(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "n"(kWaitHintNs)
+      : "memory");
+  return ok != 0;
+}
+
 // Wait for phase `parity` of `bar` to complete. Returns false (and raises the
 // CTA-wide abort flag plus the global status word) if it does not complete
 // within kWaitTimeoutNs, or if another thread of the CTA has already aborted.
@@ -80,15 +96,13 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
                                           int site) {
   if (mbar_try_wait(bar, parity)) return true;
   const unsigned long long t0 = global_ns();
-  for (uint32_t it = 1;; ++it) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((it & 63u) == 0u) {
-      if (*abort_flag) return false;
-      if (global_ns() - t0 > kWaitTimeoutNs) {
-        *abort_flag = 1;
-        atomicCAS(&g_attn_device_status, 0, kDevTimeout | (site << 8));
-        return false;
-      }
+  for (;;) {
+    if (mbar_try_wait_hint(bar, parity)) return true;
+    if (*abort_flag) return false;
+    if (global_ns() - t0 > kWaitTimeoutNs) {
+      *abort_flag = 1;
+      atomicCAS(&g_attn_device_status, 0, kDevTimeout | (site << 8));
+      return false;
     }
   }
 }
@@ -98,7 +112,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
 constexpr int kSiteDrainWait = 0x7F;
 __device__ __forceinline__ void mbar_wait_drain(uint64_t* bar, uint32_t parity) {
   const unsigned long long t0 = global_ns();
-  while (!mbar_try_wait(bar, parity)) {
+  while (!mbar_try_wait_hint(bar, parity)) {
     if (global_ns() - t0 > kWaitTimeoutNs) {
       atomicCAS(&g_attn_device_status, 0, kDevTimeout | (kSiteDrainWait << 8));
       return;
