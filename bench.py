@@ -43,7 +43,7 @@ CSRC = os.path.join(ROOT, "exact_attention_105_b200", "csrc")
 def parse_args():
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-extra", action="store_true", help="skip the forward-only target workloads")
@@ -217,6 +217,27 @@ def oracle_baseline(w, inputs, steps, per_step_s, warmup=1):
 
 # ------------------------------------------------------------------ distributed
 
+def rank_workload(w, rank: int):
+    """The shard a rank runs: the same shape, its own seed (data parallel)."""
+    return workloads.Workload(w.name, w.B, w.Hq, w.Hkv, w.N, w.d, w.causal, q_mult=w.q_mult,
+                              backward=True, seed=w.seed + rank)
+
+
+def max_over_ranks(x: float, dist, device) -> float:
+    """The slowest rank's value (a no-op for one process)."""
+    if dist is None or not dist.is_initialized() or dist.get_world_size() == 1:
+        return float(x)
+    import torch
+    t = torch.tensor([float(x)], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(flops_per_step: float, steps: int, world: int, elapsed_ms: float) -> float:
+    """Whole-job TFLOP/s: the work every rank did over the slowest rank's time."""
+    return flops_per_step * steps * world / (elapsed_ms / 1e3) / 1e12
+
+
 def dist_setup(args):
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -294,8 +315,7 @@ def run_ours(args):
                                 device_id=torch.device("cuda", local))
     w = pick_workload(args)
     fwd_only = args.mode == "fwd"
-    w_rank = workloads.Workload(w.name, w.B, w.Hq, w.Hkv, w.N, w.d, w.causal, q_mult=w.q_mult,
-                                backward=True, seed=w.seed + rank)
+    w_rank = rank_workload(w, rank)
     peaks = load_peaks()
     host = workloads.make_inputs(w_rank)
     q, k, v, do = (t.cuda() for t in host)
@@ -333,16 +353,12 @@ def run_ours(args):
     if world > 1:
         dist.barrier()
     ea.attn_check_status()
-    elapsed = ev0.elapsed_time(ev1)
-    if world > 1:
-        t = torch.tensor([elapsed], device="cuda", dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        elapsed = float(t.item())
+    elapsed = max_over_ranks(ev0.elapsed_time(ev1), dist, "cuda")
     prof = ea.profile_read()
     launches = sum(n for n, _ in prof.values())
 
     flops_step = w.fwd_flops() + (0.0 if fwd_only else w.bwd_flops())
-    value = flops_step * args.steps * world / (elapsed / 1e3) / 1e12
+    value = job_throughput(flops_step, args.steps, world, elapsed)
 
     # Roofline of the dominant kernel (largest share of the timed region).
     dom = max(prof, key=lambda kname: prof[kname][1])
@@ -398,17 +414,13 @@ def run_ours(args):
                 dst.copy_(src, non_blocking=True)
     e1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = e0.elapsed_time(e1)
-    if world > 1:
-        t = torch.tensor([e2e_ms], device="cuda", dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), dist, "cuda")
     h2d = sum(t.numel() * t.element_size() for t in pin)
     d2h = sum(t.numel() * t.element_size() for t in outs)
     if fwd_only:   # inputs q, k, v in; o and lse out
         h2d -= do.numel() * do.element_size()
         d2h = o.numel() * o.element_size() + lse.numel() * lse.element_size()
-    e2e = {"value": flops_step * e2e_steps * world / (e2e_ms / 1e3) / 1e12, "unit": UNIT,
+    e2e = {"value": job_throughput(flops_step, e2e_steps, world, e2e_ms), "unit": UNIT,
            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps}
 
     extra = None

@@ -32,6 +32,7 @@ SIGNATURES = {
     "attn_bwd_noalloc": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P,
                               _I, _I, _I, _I, _I, _F, _I, _P]),
     "attn_check_status": (_I, [_P]),
+    "attn_selftest_wait_timeout": (_I, [_P]),
     "attn_get_last_error": (ctypes.c_char_p, []),
     "attn_abi_version": (_I, []),
     "attn_profile_enable": (None, [_I]),
@@ -200,6 +201,13 @@ def profile_read():
         _check(lib.attn_profile_read(idx, ctypes.byref(name), ctypes.byref(n), ctypes.byref(ms)))
         out[name.value.decode()] = (n.value, ms.value)
     return out
+
+
+def selftest_wait_timeout(stream=None):
+    """Launch the failure-detection self-test. A kernel waits on a barrier
+    that is never signalled, gives up after two seconds, and records a timeout.
+    The next attn_check_status() raises AttnError(ATTN_ERR_TIMEOUT)."""
+    _check(load_library().attn_selftest_wait_timeout(_stream_handle(stream)))
 
 
 def attn_check_status(stream=None):

@@ -295,6 +295,23 @@ attn_status launch_bwd(const BwdArgs& a, cudaStream_t stream) {
   return ATTN_OK;
 }
 
+// ---------------------------------------------------------------- wait self-test
+// One thread waits on an mbarrier that nothing ever arrives on, through the
+// same bounded wait every pipeline role uses. The wait must give up after
+// kWaitTimeoutNs and record a timeout in the status word. This exercises the
+// failure-detection path without faulting or hanging the GPU.
+__global__ void selftest_wait_timeout_kernel() {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    attn::mbar_init(&bar, 1);
+    abort_flag = 0;
+    attn::fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) attn::mbar_wait(&bar, 0, &abort_flag, 0x7E);
+}
+
 // ---------------------------------------------------------------- static scratch
 // Backing store for attn_bwd_noalloc: the backward's lse*log2(e) and
 // rowsum(dO*O) rows live in this fixed device array instead of a
@@ -451,6 +468,16 @@ attn_status attn_bwd_noalloc(const void* q, const void* k, const void* v, const 
   BwdArgs a{mq, mk, mv, mdo, o, lse, dO, dq, dk, dv, L, Dv, B, Hq, Hkv, N, scale};
   if (d == 64) return causal ? launch_bwd<64, true>(a, stream) : launch_bwd<64, false>(a, stream);
   return causal ? launch_bwd<128, true>(a, stream) : launch_bwd<128, false>(a, stream);
+}
+
+attn_status attn_selftest_wait_timeout(attn_stream_t stream_) {
+  g_last_error[0] = '\0';
+  attn_status st = ensure_init();
+  if (st != ATTN_OK) return st;
+  selftest_wait_timeout_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream_)>>>();
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "self-test launch");
+  return ATTN_OK;
 }
 
 void attn_profile_enable(int on) {

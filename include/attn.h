@@ -140,6 +140,17 @@ attn_status attn_bwd_noalloc(const void* q, const void* k, const void* v, const 
  */
 attn_status attn_check_status(attn_stream_t stream);
 
+/*
+ * Failure-detection self-test (not an attention operation, so the pages have
+ * no counterpart). It launches one kernel on `stream` that waits on a pipeline
+ * barrier nothing ever signals, with the same bounded wait the attention
+ * kernels use. That wait gives up after two seconds and records a timeout.
+ * The next attn_check_status(stream) returns ATTN_ERR_TIMEOUT and clears the
+ * word. The GPU context stays usable. Returns ATTN_OK when the launch was
+ * queued, or ATTN_ERR_CUDA.
+ */
+attn_status attn_selftest_wait_timeout(attn_stream_t stream);
+
 /* Message of the last error on the calling thread ("" if none). The library
  * owns the string. It stays valid until the next call on the same thread. */
 const char* attn_get_last_error(void);
