@@ -17,4 +17,5 @@ from .attention_ref import (  # noqa: F401
     scores,
     softmax_rows,
     to_f64,
+    visible,
 )

@@ -16,6 +16,11 @@ written out directly and slowly so it can be checked by eye:
 * Same page, section "Von 2.0 bis 2.7": the causal mask is aligned to the
   bottom-right corner when the query and key lengths differ. Query ``i`` may
   see key ``j`` iff ``j <= i + (Nk - Nq)``. With ``Nq == Nk`` this is ``j <= i``.
+  Release 2.3 there adds sliding-window attention, and the interface section
+  lists a ``window_size`` parameter. Read plainly, with the same bottom-right
+  alignment: ``window = (left, right)`` keeps key ``j`` for query ``i`` iff
+  ``i + off - left <= j <= i + off + right`` with ``off = Nk - Nq``. A negative
+  side means unbounded. Causal is the case ``right = 0``.
 * tokenwerk.de "FlashAttention", section "Was FlashAttention veraendert", and
   unite.ai "Was ist FlashAttention?", the worked example: the method is exact,
   not an approximation. So the oracle is the definition itself. S and P are
@@ -84,21 +89,40 @@ def causal_visible(n_q: int, n_k: int) -> np.ndarray:
     return j <= i + (n_k - n_q)
 
 
+def visible(rows, n_q_total: int, n_k: int, causal: bool, window=(-1, -1)) -> np.ndarray:
+    """Boolean [len(rows), Nk]: query row i (of n_q_total) may see key j.
+
+    Bottom-right alignment with off = Nk - Nq: causal keeps j <= i + off, and
+    window (left, right) keeps i + off - left <= j <= i + off + right. A
+    negative window side is unbounded.
+    """
+    i = np.asarray(rows)[:, None]
+    j = np.arange(n_k)[None, :]
+    off = n_k - n_q_total
+    keep = np.ones((i.shape[0], n_k), dtype=bool)
+    left, right = window
+    if causal:
+        keep &= j <= i + off
+    if right >= 0:
+        keep &= j <= i + off + right
+    if left >= 0:
+        keep &= j >= i + off - left
+    return keep
+
+
 def scores(q: np.ndarray, k: np.ndarray, scale: float, causal: bool,
-           row_offset: int = 0, n_q_total: int | None = None) -> np.ndarray:
+           row_offset: int = 0, n_q_total: int | None = None, window=(-1, -1)) -> np.ndarray:
     """S = (Q K^T) * scale, with masked entries set to -inf.
 
     ``q`` holds query rows ``row_offset .. row_offset + len(q)`` of a sequence
     of ``n_q_total`` queries (default: just these rows). That is how the
-    row-chunked and row-sampled callers keep the causal mask right.
+    row-chunked and row-sampled callers keep the causal/window mask right.
     """
     s = (q @ k.T) * scale
-    if causal:
+    if causal or window[0] >= 0 or window[1] >= 0:
         n_q_total = q.shape[0] if n_q_total is None else n_q_total
-        n_k = k.shape[0]
-        rows = np.arange(row_offset, row_offset + q.shape[0])[:, None]
-        cols = np.arange(n_k)[None, :]
-        s = np.where(cols <= rows + (n_k - n_q_total), s, -np.inf)
+        rows = np.arange(row_offset, row_offset + q.shape[0])
+        s = np.where(visible(rows, n_q_total, k.shape[0], causal, window), s, -np.inf)
     return s
 
 
@@ -116,14 +140,15 @@ def softmax_rows(s: np.ndarray):
     return p, m, l
 
 
-def attention_head(q, k, v, scale: float, causal: bool, row_chunk: int = ROW_CHUNK):
+def attention_head(q, k, v, scale: float, causal: bool, row_chunk: int = ROW_CHUNK,
+                   window=(-1, -1)):
     """O and lse for one (query head, KV head) pair; q [Nq,d], k/v [Nk,d] float64."""
     n_q = q.shape[0]
     o = np.empty((n_q, v.shape[1]), dtype=np.float64)
     lse = np.empty(n_q, dtype=np.float64)
     for r0 in range(0, n_q, row_chunk):
         r1 = min(n_q, r0 + row_chunk)
-        s = scores(q[r0:r1], k, scale, causal, row_offset=r0, n_q_total=n_q)
+        s = scores(q[r0:r1], k, scale, causal, row_offset=r0, n_q_total=n_q, window=window)
         p, m, l = softmax_rows(s)
         o[r0:r1] = p @ v
         with np.errstate(divide="ignore"):
@@ -131,22 +156,22 @@ def attention_head(q, k, v, scale: float, causal: bool, row_chunk: int = ROW_CHU
     return o, lse
 
 
-def attention_head_rows(q_rows, k, v, scale: float, causal: bool, rows, n_q_total: int):
+def attention_head_rows(q_rows, k, v, scale: float, causal: bool, rows, n_q_total: int,
+                        window=(-1, -1)):
     """O and lse for selected query rows (indices ``rows`` of ``n_q_total``)."""
     rows = np.asarray(rows)
     s = (q_rows @ k.T) * scale
-    if causal:
-        cols = np.arange(k.shape[0])[None, :]
-        s = np.where(cols <= rows[:, None] + (k.shape[0] - n_q_total), s, -np.inf)
+    if causal or window[0] >= 0 or window[1] >= 0:
+        s = np.where(visible(rows, n_q_total, k.shape[0], causal, window), s, -np.inf)
     p, m, l = softmax_rows(s)
     with np.errstate(divide="ignore"):
         lse = np.where(l > 0, m + np.log(np.where(l > 0, l, 1.0)), -np.inf)
     return p @ v, lse
 
 
-def attention_head_bwd(q, k, v, do, scale: float, causal: bool):
+def attention_head_bwd(q, k, v, do, scale: float, causal: bool, window=(-1, -1)):
     """dQ, dK, dV for one head pair, from explicit S and P (no recompute trick)."""
-    s = scores(q, k, scale, causal)
+    s = scores(q, k, scale, causal, window=window)
     p, _, _ = softmax_rows(s)
     dv = p.T @ do
     dp = do @ v.T
@@ -167,8 +192,8 @@ def _kv_head(hq: int, n_q_heads: int, n_kv_heads: int) -> int:
     return hq // (n_q_heads // n_kv_heads)
 
 
-def attention_forward(q, k, v, scale: float, causal: bool):
-    """O [B,Hq,Nq,d] and lse [B,Hq,Nq] in float64."""
+def attention_forward(q, k, v, scale: float, causal: bool, window=(-1, -1)):
+    """O [B,Hq,Nq,d] and lse [B,Hq,Nq] in float64 (K/V may have Nk != Nq rows)."""
     q, k, v = to_f64(q), to_f64(k), to_f64(v)
     B, Hq, Nq, _ = q.shape
     Hkv = k.shape[1]
@@ -177,21 +202,23 @@ def attention_forward(q, k, v, scale: float, causal: bool):
     for b in range(B):
         for h in range(Hq):
             hk = _kv_head(h, Hq, Hkv)
-            o[b, h], lse[b, h] = attention_head(q[b, h], k[b, hk], v[b, hk], scale, causal)
+            o[b, h], lse[b, h] = attention_head(q[b, h], k[b, hk], v[b, hk], scale, causal,
+                                                window=window)
     return o, lse
 
 
-def attention_forward_rows(q, k, v, scale: float, causal: bool, b: int, hq: int, rows):
+def attention_forward_rows(q, k, v, scale: float, causal: bool, b: int, hq: int, rows,
+                           window=(-1, -1)):
     """O and lse of the listed query rows of head (b, hq), for full-size spot checks."""
     Hq, Nq = q.shape[1], q.shape[2]
     hk = _kv_head(hq, Hq, k.shape[1])
     rows = np.asarray(rows)
     q_rows = to_f64(q[b, hq][rows])
     return attention_head_rows(q_rows, to_f64(k[b, hk]), to_f64(v[b, hk]), scale, causal,
-                               rows, Nq)
+                               rows, Nq, window=window)
 
 
-def attention_backward(q, k, v, do, scale: float, causal: bool, heads=None):
+def attention_backward(q, k, v, do, scale: float, causal: bool, heads=None, window=(-1, -1)):
     """dQ [B,Hq,N,d], dK and dV [B,Hkv,N,d] in float64.
 
     ``heads``: optional list of (b, hkv) KV heads to compute (the others are
@@ -212,7 +239,8 @@ def attention_backward(q, k, v, do, scale: float, causal: bool, heads=None):
         dk[b, hk] = 0.0
         dv[b, hk] = 0.0
         for h in range(hk * G, (hk + 1) * G):
-            gq, gk, gv = attention_head_bwd(q[b, h], k[b, hk], v[b, hk], do[b, h], scale, causal)
+            gq, gk, gv = attention_head_bwd(q[b, h], k[b, hk], v[b, hk], do[b, h], scale, causal,
+                                            window=window)
             dq[b, h] = gq
             dk[b, hk] += gk
             dv[b, hk] += gv
@@ -230,7 +258,7 @@ def attention_backward(q, k, v, do, scale: float, causal: bool, heads=None):
 # --------------------------------------------------------------------------
 
 def online_softmax_attention_head(q, k, v, scale: float, causal: bool, block: int,
-                                  rescale_threshold: float = 0.0):
+                                  rescale_threshold: float = 0.0, window=(-1, -1)):
     """One head, keys visited in blocks of ``block`` with a running max and sum.
 
     ``rescale_threshold`` (natural-log units) lets the running max lag the
@@ -243,7 +271,7 @@ def online_softmax_attention_head(q, k, v, scale: float, causal: bool, block: in
     m = np.full(n_q, -np.inf)
     l = np.zeros(n_q)
     acc = np.zeros((n_q, v.shape[1]))
-    vis = causal_visible(n_q, n_k) if causal else np.ones((n_q, n_k), dtype=bool)
+    vis = visible(np.arange(n_q), n_q, n_k, causal, window)
     for c0 in range(0, n_k, block):
         c1 = min(n_k, c0 + block)
         s = (q @ k[c0:c1].T) * scale
@@ -271,7 +299,7 @@ def online_softmax_attention_head(q, k, v, scale: float, causal: bool, block: in
 # Brute force for tiny inputs: scalar loops and math.exp, nothing vectorised.
 # --------------------------------------------------------------------------
 
-def attention_bruteforce(q, k, v, scale: float, causal: bool):
+def attention_bruteforce(q, k, v, scale: float, causal: bool, window=(-1, -1)):
     """Pure-Python O and lse for one head; q [Nq][d], k/v [Nk][d] nested lists."""
     n_q, n_k, d_v = len(q), len(k), len(v[0])
     out, lses = [], []
@@ -279,6 +307,10 @@ def attention_bruteforce(q, k, v, scale: float, causal: bool):
         logits = []
         for j in range(n_k):
             if causal and j > i + (n_k - n_q):
+                continue
+            if window[1] >= 0 and j > i + (n_k - n_q) + window[1]:
+                continue
+            if window[0] >= 0 and j < i + (n_k - n_q) - window[0]:
                 continue
             dot = 0.0
             for c in range(len(q[i])):

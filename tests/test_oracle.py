@@ -308,3 +308,78 @@ def test_backward_mutant_without_row_dot_is_caught():
     dq_bad = 0.8 * ((p * (do @ v.T)) @ k)
     dq, _, _ = ref.attention_head_bwd(q, k, v, do, 0.8, False)
     assert np.max(np.abs(dq_bad - dq)) > 1e-3
+
+
+# ------------------------------------------- sliding window and Nq != Nk
+# hysenlabs.com, 'Von 2.0 bis 2.7': sliding-window attention (2.3) and the
+# bottom-right causal alignment for Nq != Nk (2.1).
+
+def test_window_reduces_to_known_masks():
+    n = 50
+    q, k, v = rand(n, 8), rand(n, 8), rand(n, 8)
+    full = oracle.attention_head(q, k, v, 0.5, False)
+    causal = oracle.attention_head(q, k, v, 0.5, True)
+    wide = oracle.attention_head(q, k, v, 0.5, False, window=(n, n))
+    left_only = oracle.attention_head(q, k, v, 0.5, False, window=(n, 0))
+    for a, b in ((full, wide), (causal, left_only)):
+        np.testing.assert_allclose(a[0], b[0], rtol=0, atol=1e-14)
+        np.testing.assert_allclose(a[1], b[1], rtol=0, atol=1e-14)
+
+
+def test_window_zero_is_identity_on_v():
+    """window (0, 0) with Nq == Nk: each query sees only its own key, so O = V."""
+    n = 20
+    q, k, v = rand(n, 4), rand(n, 4), rand(n, 3)
+    o, lse = oracle.attention_head(q, k, v, 0.7, False, window=(0, 0))
+    np.testing.assert_allclose(o, v, rtol=0, atol=1e-15)
+    np.testing.assert_allclose(lse, 0.7 * np.sum(q * k, axis=1), rtol=0, atol=1e-14)
+
+
+def test_visible_counts_closed_form():
+    """With Nq == Nk == n, window (l, r): row i sees min(i, l) + 1 + min(n-1-i, r) keys."""
+    n, l, r = 30, 5, 3
+    vis = oracle.visible(np.arange(n), n, n, False, (l, r))
+    expect = [min(i, l) + 1 + min(n - 1 - i, r) for i in range(n)]
+    assert vis.sum(axis=1).tolist() == expect
+
+
+@pytest.mark.parametrize("window", [(2, 1), (0, 3), (3, -1), (-1, 2)])
+@pytest.mark.parametrize("nq,nk,causal", [(5, 5, False), (4, 6, True), (6, 4, True), (3, 7, False)])
+def test_window_bruteforce(window, nq, nk, causal):
+    q, k, v = rand(nq, 3), rand(nk, 3), rand(nk, 2)
+    o, lse = oracle.attention_head(q, k, v, 0.9, causal, window=window)
+    ob, lb = oracle.attention_bruteforce(q.tolist(), k.tolist(), v.tolist(), 0.9, causal, window)
+    np.testing.assert_allclose(o, np.array(ob), rtol=0, atol=1e-14)
+    np.testing.assert_allclose(lse, np.array(lb), rtol=0, atol=1e-14)
+
+
+@pytest.mark.parametrize("nq,nk,causal,window", [(40, 70, True, (-1, -1)), (70, 40, True, (-1, -1)),
+                                                 (50, 50, False, (7, 3)), (33, 61, True, (9, -1))])
+def test_masked_forward_and_backward_match_torch(nq, nk, causal, window):
+    """Library routine: torch float64 SDPA with the explicit boolean mask, and its autograd."""
+    q = torch.randn(1, 2, nq, 8, dtype=torch.float64, requires_grad=True)
+    k = torch.randn(1, 2, nk, 8, dtype=torch.float64, requires_grad=True)
+    v = torch.randn(1, 2, nk, 8, dtype=torch.float64, requires_grad=True)
+    do = torch.randn(1, 2, nq, 8, dtype=torch.float64)
+    mask = torch.from_numpy(oracle.visible(np.arange(nq), nq, nk, causal, window))
+    rows_ok = mask.any(dim=1)
+    out = torch.nn.functional.scaled_dot_product_attention(q, k, v, attn_mask=mask, scale=0.3)
+    out = torch.where(rows_ok[None, None, :, None], out, torch.zeros_like(out))
+    (out * do).sum().backward()
+    o, lse = oracle.attention_forward(q.detach(), k.detach(), v.detach(), 0.3, causal, window=window)
+    np.testing.assert_allclose(o, out.detach().numpy(), rtol=0, atol=1e-12)
+    assert np.all(np.isneginf(lse[..., ~rows_ok.numpy()]))
+    dq, dk, dv = oracle.attention_backward(q.detach(), k.detach(), v.detach(), do, 0.3, causal,
+                                           window=window)
+    np.testing.assert_allclose(dq, q.grad.numpy(), rtol=0, atol=1e-12)
+    np.testing.assert_allclose(dk, k.grad.numpy(), rtol=0, atol=1e-12)
+    np.testing.assert_allclose(dv, v.grad.numpy(), rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("window", [(0, 0), (4, 2), (10, -1)])
+def test_online_softmax_with_window(window):
+    q, k, v = rand(60, 8), rand(60, 8), rand(60, 8)
+    o1, l1 = oracle.attention_head(q, k, v, 0.5, False, window=window)
+    o2, l2 = oracle.online_softmax_attention_head(q, k, v, 0.5, False, 16, 8 * math.log(2), window)
+    np.testing.assert_allclose(o2, o1, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(l2, l1, rtol=0, atol=1e-12)
