@@ -6,8 +6,10 @@ current CUDA stream from torch tensors and calls the C ABI declared in
 is no fallback: if the shared library is missing or the device is not an
 sm_100 part, every call raises.
 
-Layout: q, o, dO, dq are [B, Hq, N, d]. k, v, dk, dv are [B, Hkv, N, d].
-All are contiguous bfloat16 CUDA tensors. lse is [B, Hq, N] float32.
+Layout: q, o, dO, dq are [B, Hq, Nq, d]. k, v, dk, dv are [B, Hkv, Nk, d].
+All are contiguous bfloat16 CUDA tensors. lse is [B, Hq, Nq] float32.
+``attn_fwd``/``attn_bwd`` need Nq == Nk; the ``*_masked`` calls take
+Nq != Nk (bottom-right causal alignment) and a sliding window.
 """
 from __future__ import annotations
 
@@ -31,6 +33,9 @@ SIGNATURES = {
     "attn_bwd_workspace_size": (_SZ, [_I, _I, _I, _I]),
     "attn_bwd_noalloc": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P,
                               _I, _I, _I, _I, _I, _F, _I, _P]),
+    "attn_fwd_masked": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _I, _I, _I, _P]),
+    "attn_bwd_masked": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _SZ,
+                             _I, _I, _I, _I, _I, _I, _F, _I, _I, _I, _P]),
     "attn_check_status": (_I, [_P]),
     "attn_selftest_wait_timeout": (_I, [_P]),
     "attn_get_last_error": (ctypes.c_char_p, []),
@@ -178,6 +183,74 @@ def attn_bwd_noalloc(q, k, v, o, lse, dO, dq, dk, dv, scale=None, causal=False, 
                                 _dev_ptr(dq, "dq"), _dev_ptr(dk, "dk"), _dev_ptr(dv, "dv"),
                                 B, Hq, Hkv, N, d, scale, int(bool(causal)),
                                 _stream_handle(stream)))
+    return dq, dk, dv
+
+
+def _window(window):
+    left, right = (int(window[0]), int(window[1]))
+    return max(left, -1), max(right, -1)
+
+
+def attn_fwd_masked(q, k, v, o=None, lse=None, scale=None, causal=False, window=(-1, -1),
+                    stream=None):
+    """Forward with Nq = q.shape[2] queries, Nk = k.shape[2] keys and a sliding
+    window (left, right); a negative side is unbounded. Query i sees key j iff
+    i + Nk - Nq - left <= j <= i + Nk - Nq + right (and j <= i + Nk - Nq when
+    causal). Rows that see no key get o = 0, lse = -inf. Returns (o, lse)."""
+    import torch
+    B, Hq, Nq, d = q.shape
+    Hkv, Nk = k.shape[1], k.shape[2]
+    if k.shape != (B, Hkv, Nk, d) or v.shape != k.shape:
+        raise ValueError(f"k/v shape {tuple(k.shape)}/{tuple(v.shape)} does not match q {tuple(q.shape)}")
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _check_dtype(t, torch.bfloat16, n)
+    o = torch.empty_like(q) if o is None else o
+    lse = torch.empty((B, Hq, Nq), dtype=torch.float32, device=q.device) if lse is None else lse
+    _check_dtype(o, torch.bfloat16, "o")
+    _check_dtype(lse, torch.float32, "lse")
+    if o.shape != q.shape or lse.shape != (B, Hq, Nq):
+        raise ValueError("o/lse shape mismatch")
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    wl, wr = _window(window)
+    lib = load_library()
+    _check(lib.attn_fwd_masked(_dev_ptr(q, "q"), _dev_ptr(k, "k"), _dev_ptr(v, "v"),
+                               _dev_ptr(o, "o"), _dev_ptr(lse, "lse"), B, Hq, Hkv, Nq, Nk, d,
+                               scale, int(bool(causal)), wl, wr, _stream_handle(stream)))
+    return o, lse
+
+
+def attn_bwd_masked(q, k, v, o, lse, dO, dq=None, dk=None, dv=None, workspace=None, scale=None,
+                    causal=False, window=(-1, -1), stream=None):
+    """Backward of attn_fwd_masked with the same causal/window; returns (dq, dk, dv)."""
+    import torch
+    B, Hq, Nq, d = q.shape
+    Hkv, Nk = k.shape[1], k.shape[2]
+    if k.shape != (B, Hkv, Nk, d) or v.shape != k.shape or o.shape != q.shape \
+            or dO.shape != q.shape or lse.shape != (B, Hq, Nq):
+        raise ValueError("shape mismatch among q, k, v, o, lse, dO")
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (o, "o"), (dO, "dO")):
+        _check_dtype(t, torch.bfloat16, n)
+    _check_dtype(lse, torch.float32, "lse")
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    for t, n, ref in ((dq, "dq", q), (dk, "dk", k), (dv, "dv", v)):
+        _check_dtype(t, torch.bfloat16, n)
+        if t.shape != ref.shape:
+            raise ValueError(f"{n} shape mismatch")
+    need = attn_bwd_workspace_size(B, Hq, Nq, d)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    wl, wr = _window(window)
+    lib = load_library()
+    _check(lib.attn_bwd_masked(_dev_ptr(q, "q"), _dev_ptr(k, "k"), _dev_ptr(v, "v"),
+                               _dev_ptr(o, "o"), _dev_ptr(lse, "lse"), _dev_ptr(dO, "dO"),
+                               _dev_ptr(dq, "dq"), _dev_ptr(dk, "dk"), _dev_ptr(dv, "dv"),
+                               _dev_ptr(workspace, "workspace"),
+                               workspace.numel() * workspace.element_size(),
+                               B, Hq, Hkv, Nq, Nk, d, scale, int(bool(causal)), wl, wr,
+                               _stream_handle(stream)))
     return dq, dk, dv
 
 

@@ -196,12 +196,31 @@ attn_status check_shape(int B, int Hq, int Hkv, int N, int d, float scale, bool*
   return ATTN_OK;
 }
 
-template <int D, bool CAUSAL>
+// Which keys each query row sees: the three kernel mask modes and the window
+// bounds they use. window_left/right < 0 is unbounded; causal caps the right
+// side at 0. Same-length problems without a left window keep the unmasked
+// and causal fast paths.
+struct MaskSpec {
+  int mode;
+  attn::KeyWindow win;
+};
+
+MaskSpec mask_spec(int Nq, int Nk, int causal, int window_left, int window_right) {
+  using namespace attn;
+  const int wl = window_left < 0 ? kUnbounded : std::min(window_left, kUnbounded);
+  int wr = window_right < 0 ? kUnbounded : std::min(window_right, kUnbounded);
+  if (causal) wr = 0;
+  const bool plain = Nq == Nk && wl == kUnbounded && (causal || wr == kUnbounded);
+  const int mode = plain ? (causal ? kMaskCausal : kMaskNone) : kMaskGeneral;
+  return MaskSpec{mode, KeyWindow{Nk - Nq, wl, wr}};
+}
+
+template <int D, int MODE>
 attn_status launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
-                       void* o, float* lse, int B, int Hq, int Hkv, int N, float scale,
-                       cudaStream_t stream) {
+                       void* o, float* lse, int B, int Hq, int Hkv, int Nq, int Nk, float scale,
+                       attn::KeyWindow win, cudaStream_t stream) {
   using Cfg = attn::FwdCfg<D>;
-  auto kern = attn::fwd_kernel<D, CAUSAL>;
+  auto kern = attn::fwd_kernel<D, MODE>;
   static std::once_flag attr_once;
   static cudaError_t attr_err = cudaSuccess;
   static int launch_regs = 0;
@@ -218,13 +237,13 @@ attn_status launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUten
   if (launch_regs != attn::kFwdRegsLaunch)
     return fail(ATTN_ERR_CUDA, "fwd kernel built with %d registers/thread, expected %d",
                 launch_regs, attn::kFwdRegsLaunch);
-  const long long blocks = static_cast<long long>(B) * Hq * ((N + 255) / 256);
+  const long long blocks = static_cast<long long>(B) * Hq * ((Nq + 255) / 256);
   if (blocks > 0x7FFFFFFFLL) return fail(ATTN_ERR_ARG, "problem too large for one launch");
   dim3 grid(static_cast<unsigned>(blocks));
   const float scale_log2 = scale * 1.4426950408889634f;
   ProfScope ps(kProfFwd, stream);
   kern<<<grid, Cfg::kThreads, Cfg::kSmemAlloc, stream>>>(
-      mq, mk, mv, static_cast<__nv_bfloat16*>(o), lse, Hq, Hq / Hkv, N, scale_log2);
+      mq, mk, mv, static_cast<__nv_bfloat16*>(o), lse, Hq, Hq / Hkv, Nq, Nk, scale_log2, win);
   ps.end();
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "fwd kernel launch");
@@ -247,34 +266,34 @@ struct BwdArgs {
   const void* dO;
   void *dq, *dk, *dv;
   float *L, *Dv;
-  int B, Hq, Hkv, N;
+  int B, Hq, Hkv, Nq, Nk;
   float scale;
+  attn::KeyWindow win;
 };
 
-template <int D, bool CAUSAL>
+template <int D, int MODE>
 attn_status launch_bwd(const BwdArgs& a, cudaStream_t stream) {
   using namespace attn;
-  const int Npad = pad128(a.N);
-  const int nblk = Npad / 128;
+  const int Npad = pad128(a.Nq);
   const int group = a.Hq / a.Hkv;
   const float scale_log2 = a.scale * kLog2e;
 
   const long long rows = static_cast<long long>(a.B) * a.Hq * Npad;
-  const long long g1 = static_cast<long long>(nblk) * a.B * a.Hkv;
-  const long long g2 = static_cast<long long>(nblk) * a.B * a.Hq;
+  const long long g1 = static_cast<long long>(pad128(a.Nk) / 128) * a.B * a.Hkv;
+  const long long g2 = static_cast<long long>(Npad / 128) * a.B * a.Hq;
   if (rows / 32 > 0x7FFFFFFFLL) return fail(ATTN_ERR_ARG, "problem too large for one launch");
   ProfScope p0(kProfBwdPre, stream);
   bwd_pre_kernel<D><<<static_cast<unsigned>(rows / 32), 256, 0, stream>>>(
       static_cast<const __nv_bfloat16*>(a.o), static_cast<const __nv_bfloat16*>(a.dO), a.lse,
-      a.L, a.Dv, a.N, Npad);
+      a.L, a.Dv, a.Nq, Npad);
   p0.end();
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "bwd preprocess launch");
 
   static std::once_flag o1, o2;
   static cudaError_t e1 = cudaSuccess, e2 = cudaSuccess;
-  auto k1 = bwd_dkdv_kernel<D, CAUSAL>;
-  auto k2 = bwd_dq_kernel<D, CAUSAL>;
+  auto k1 = bwd_dkdv_kernel<D, MODE>;
+  auto k2 = bwd_dq_kernel<D, MODE>;
   if ((e = set_smem_once(k1, DkdvCfg<D>::kSmemAlloc, o1, e1)) != cudaSuccess)
     return cuda_fail(e, "cudaFuncSetAttribute(dkdv)");
   if ((e = set_smem_once(k2, DqCfg<D>::kSmemAlloc, o2, e2)) != cudaSuccess)
@@ -283,13 +302,14 @@ attn_status launch_bwd(const BwdArgs& a, cudaStream_t stream) {
   ProfScope p1(kProfBwdDkdv, stream);
   k1<<<dim3(static_cast<unsigned>(g1)), DkdvCfg<D>::kThreads, DkdvCfg<D>::kSmemAlloc, stream>>>(
       a.mq, a.mk, a.mv, a.mdo, a.L, a.Dv, static_cast<__nv_bfloat16*>(a.dk),
-      static_cast<__nv_bfloat16*>(a.dv), a.Hq, group, a.N, Npad, scale_log2, a.scale);
+      static_cast<__nv_bfloat16*>(a.dv), a.Hq, group, a.Nq, a.Nk, Npad, scale_log2, a.scale,
+      a.win);
   p1.end();
   if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "bwd dK/dV launch");
   ProfScope p2(kProfBwdDq, stream);
   k2<<<dim3(static_cast<unsigned>(g2)), DqCfg<D>::kThreads, DqCfg<D>::kSmemAlloc, stream>>>(
-      a.mq, a.mk, a.mv, a.mdo, a.L, a.Dv, static_cast<__nv_bfloat16*>(a.dq), a.Hq, group, a.N,
-      Npad, scale_log2, a.scale);
+      a.mq, a.mk, a.mv, a.mdo, a.L, a.Dv, static_cast<__nv_bfloat16*>(a.dq), a.Hq, group, a.Nq,
+      a.Nk, Npad, scale_log2, a.scale, a.win);
   p2.end();
   if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "bwd dQ launch");
   return ATTN_OK;
@@ -346,42 +366,180 @@ attn_status static_scratch_ptr(void** out) {
   return ATTN_OK;
 }
 
+// Rows of a problem with no keys: lse = -inf.
+__global__ void fill_neg_inf_kernel(float* p, long long n) {
+  for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < n;
+       i += static_cast<long long>(gridDim.x) * blockDim.x)
+    p[i] = -INFINITY;
+}
+
+template <int D>
+attn_status dispatch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                         void* o, float* lse, int B, int Hq, int Hkv, int Nq, int Nk, float scale,
+                         const MaskSpec& m, cudaStream_t stream) {
+  using namespace attn;
+  if (m.mode == kMaskNone)
+    return launch_fwd<D, kMaskNone>(mq, mk, mv, o, lse, B, Hq, Hkv, Nq, Nk, scale, m.win, stream);
+  if (m.mode == kMaskCausal)
+    return launch_fwd<D, kMaskCausal>(mq, mk, mv, o, lse, B, Hq, Hkv, Nq, Nk, scale, m.win,
+                                      stream);
+  return launch_fwd<D, kMaskGeneral>(mq, mk, mv, o, lse, B, Hq, Hkv, Nq, Nk, scale, m.win, stream);
+}
+
+template <int D>
+attn_status dispatch_bwd(const BwdArgs& a, int mode, cudaStream_t stream) {
+  using namespace attn;
+  if (mode == kMaskNone) return launch_bwd<D, kMaskNone>(a, stream);
+  if (mode == kMaskCausal) return launch_bwd<D, kMaskCausal>(a, stream);
+  return launch_bwd<D, kMaskGeneral>(a, stream);
+}
+
+attn_status check_common(int B, int Hq, int Hkv, int Nq, int Nk, int d, float scale, int causal,
+                         bool* no_rows, bool* no_keys) {
+  bool eq = false, ek = false;
+  attn_status st = check_shape(B, Hq, Hkv, Nq, d, scale, &eq);
+  if (st != ATTN_OK) return st;
+  if ((st = check_shape(B, Hq, Hkv, Nk, d, scale, &ek)) != ATTN_OK) return st;
+  if (causal != 0 && causal != 1) return fail(ATTN_ERR_ARG, "causal must be 0 or 1");
+  *no_rows = eq;
+  *no_keys = ek;
+  return ATTN_OK;
+}
+
+attn_status check_args(const void* const* ptrs, const char* const* names, const bool* used,
+                       int n) {
+  for (int i = 0; i < n; ++i) {
+    if (!used[i]) continue;
+    if (ptrs[i] == nullptr) return fail(ATTN_ERR_ARG, "%s is null", names[i]);
+    if (!aligned16(ptrs[i])) return fail(ATTN_ERR_ARG, "%s is not 16-byte aligned", names[i]);
+  }
+  return ATTN_OK;
+}
+
+attn_status check_used_ptrs(const void* const* ptrs, const char* const* names, const bool* used,
+                            int n) {
+  const void* p[16];
+  const char* nm[16];
+  int m = 0;
+  for (int i = 0; i < n && m < 16; ++i)
+    if (used[i]) {
+      p[m] = ptrs[i];
+      nm[m++] = names[i];
+    }
+  return check_ptrs(p, nm, m);
+}
+
+attn_status fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                     int Hq, int Hkv, int Nq, int Nk, int d, float scale, int causal,
+                     int window_left, int window_right, cudaStream_t stream) {
+  g_last_error[0] = '\0';
+  bool no_rows = false, no_keys = false;
+  attn_status st = check_common(B, Hq, Hkv, Nq, Nk, d, scale, causal, &no_rows, &no_keys);
+  if (st != ATTN_OK) return st;
+  if (no_rows) return ATTN_OK;                 // B == 0 or Nq == 0: nothing to write
+  const void* ptrs[5] = {q, k, v, o, lse};
+  const char* names[5] = {"q", "k", "v", "o", "lse"};
+  const bool used[5] = {!no_keys, !no_keys, !no_keys, true, true};
+  if ((st = check_args(ptrs, names, used, 5)) != ATTN_OK) return st;
+  if ((st = ensure_init()) != ATTN_OK) return st;
+  if ((st = check_used_ptrs(ptrs, names, used, 5)) != ATTN_OK) return st;
+  if (no_keys) {
+    // Nk == 0: every row sees no key, so O = 0 and lse = -inf.
+    const long long rows = static_cast<long long>(B) * Hq * Nq;
+    cudaError_t e = cudaMemsetAsync(o, 0, static_cast<size_t>(rows) * d * 2, stream);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(o)");
+    fill_neg_inf_kernel<<<static_cast<unsigned>(std::min<long long>((rows + 255) / 256, 4096)),
+                          256, 0, stream>>>(lse, rows);
+    if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "lse fill launch");
+    return ATTN_OK;
+  }
+  CUtensorMap mq, mk, mv;
+  if ((st = make_map(&mq, q, d, Nq, B * Hq)) != ATTN_OK) return st;
+  if ((st = make_map(&mk, k, d, Nk, B * Hkv)) != ATTN_OK) return st;
+  if ((st = make_map(&mv, v, d, Nk, B * Hkv)) != ATTN_OK) return st;
+  const MaskSpec m = mask_spec(Nq, Nk, causal, window_left, window_right);
+  if (d == 64) return dispatch_fwd<64>(mq, mk, mv, o, lse, B, Hq, Hkv, Nq, Nk, scale, m, stream);
+  return dispatch_fwd<128>(mq, mk, mv, o, lse, B, Hq, Hkv, Nq, Nk, scale, m, stream);
+}
+
+// Backward shared by attn_bwd, attn_bwd_masked and attn_bwd_noalloc. With
+// use_static the scratch rows live in g_bwd_scratch instead of `workspace`.
+attn_status bwd_impl(const void* q, const void* k, const void* v, const void* o,
+                     const float* lse, const void* dO, void* dq, void* dk, void* dv,
+                     void* workspace, size_t workspace_bytes, bool use_static, int B, int Hq,
+                     int Hkv, int Nq, int Nk, int d, float scale, int causal, int window_left,
+                     int window_right, cudaStream_t stream) {
+  g_last_error[0] = '\0';
+  bool no_rows = false, no_keys = false;
+  attn_status st = check_common(B, Hq, Hkv, Nq, Nk, d, scale, causal, &no_rows, &no_keys);
+  if (st != ATTN_OK) return st;
+  if (B == 0 || (no_rows && no_keys)) return ATTN_OK;
+  const void* ptrs[10] = {q, k, v, o, lse, dO, dq, dk, dv, workspace};
+  const char* names[10] = {"q", "k", "v", "o", "lse", "dO", "dq", "dk", "dv", "workspace"};
+  const bool work = !no_rows && !no_keys;
+  const bool used[10] = {work, work, work, work, work, work, !no_rows, !no_keys, !no_keys,
+                         work && !use_static};
+  if ((st = check_args(ptrs, names, used, 10)) != ATTN_OK) return st;
+  const size_t need = attn_bwd_workspace_size(B, Hq, Nq, d);
+  if (work && use_static && need > kStaticScratchBytes)
+    return fail(ATTN_ERR_ARG,
+                "attn_bwd_noalloc: this shape needs %zu bytes of scratch, but the static area "
+                "holds %zu (B*Hq*ceil128(N) must be <= %zu); use attn_bwd with a workspace",
+                need, kStaticScratchBytes, kStaticScratchBytes / (2 * sizeof(float)));
+  if (work && !use_static && workspace_bytes < need)
+    return fail(ATTN_ERR_ARG, "workspace is %zu bytes, needs %zu", workspace_bytes, need);
+  if ((st = ensure_init()) != ATTN_OK) return st;
+  if ((st = check_used_ptrs(ptrs, names, used, 10)) != ATTN_OK) return st;
+  if (!work) {
+    // No keys: dQ = 0. No queries: dK = dV = 0. (The other side is empty.)
+    const size_t kv_bytes = static_cast<size_t>(B) * Hkv * Nk * d * 2;
+    const size_t q_bytes = static_cast<size_t>(B) * Hq * Nq * d * 2;
+    cudaError_t e = cudaSuccess;
+    if (!no_rows) e = cudaMemsetAsync(dq, 0, q_bytes, stream);
+    if (e == cudaSuccess && !no_keys) e = cudaMemsetAsync(dk, 0, kv_bytes, stream);
+    if (e == cudaSuccess && !no_keys) e = cudaMemsetAsync(dv, 0, kv_bytes, stream);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(gradients)");
+    return ATTN_OK;
+  }
+  void* scratch = workspace;
+  if (use_static && (st = static_scratch_ptr(&scratch)) != ATTN_OK) return st;
+  CUtensorMap mq, mk, mv, mdo;
+  if ((st = make_map(&mq, q, d, Nq, B * Hq)) != ATTN_OK) return st;
+  if ((st = make_map(&mk, k, d, Nk, B * Hkv)) != ATTN_OK) return st;
+  if ((st = make_map(&mv, v, d, Nk, B * Hkv)) != ATTN_OK) return st;
+  if ((st = make_map(&mdo, dO, d, Nq, B * Hq)) != ATTN_OK) return st;
+  // The preprocess kernel writes every scratch row the other two kernels
+  // read, so nothing left from an earlier call is ever used and no clearing
+  // is needed (this matters for the static area).
+  float* L = static_cast<float*>(scratch);
+  float* Dv = L + static_cast<size_t>(B) * Hq * attn::pad128(Nq);
+  const MaskSpec m = mask_spec(Nq, Nk, causal, window_left, window_right);
+  BwdArgs a{mq, mk, mv, mdo, o, lse, dO, dq, dk, dv, L, Dv, B, Hq, Hkv, Nq, Nk, scale, m.win};
+  if (d == 64) return dispatch_bwd<64>(a, m.mode, stream);
+  return dispatch_bwd<128>(a, m.mode, stream);
+}
+
 }  // namespace
 
 extern "C" {
 
-int attn_abi_version(void) { return 100; }
+int attn_abi_version(void) { return 101; }
 
 const char* attn_get_last_error(void) { return g_last_error; }
 
 attn_status attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B,
                      int Hq, int Hkv, int N, int d, float scale, int causal,
                      attn_stream_t stream_) {
-  g_last_error[0] = '\0';
-  bool empty = false;
-  attn_status st = check_shape(B, Hq, Hkv, N, d, scale, &empty);
-  if (st != ATTN_OK) return st;
-  if (causal != 0 && causal != 1) return fail(ATTN_ERR_ARG, "causal must be 0 or 1");
-  if (empty) return ATTN_OK;
-  const void* ptrs[5] = {q, k, v, o, lse};
-  const char* names[5] = {"q", "k", "v", "o", "lse"};
-  for (int i = 0; i < 5; ++i) {
-    if (ptrs[i] == nullptr) return fail(ATTN_ERR_ARG, "%s is null", names[i]);
-    if (!aligned16(ptrs[i])) return fail(ATTN_ERR_ARG, "%s is not 16-byte aligned", names[i]);
-  }
-  st = ensure_init();
-  if (st != ATTN_OK) return st;
-  if ((st = check_ptrs(ptrs, names, 5)) != ATTN_OK) return st;
-  cudaStream_t stream = static_cast<cudaStream_t>(stream_);
-  CUtensorMap mq, mk, mv;
-  if ((st = make_map(&mq, q, d, N, B * Hq)) != ATTN_OK) return st;
-  if ((st = make_map(&mk, k, d, N, B * Hkv)) != ATTN_OK) return st;
-  if ((st = make_map(&mv, v, d, N, B * Hkv)) != ATTN_OK) return st;
-  if (d == 64)
-    return causal ? launch_fwd<64, true>(mq, mk, mv, o, lse, B, Hq, Hkv, N, scale, stream)
-                  : launch_fwd<64, false>(mq, mk, mv, o, lse, B, Hq, Hkv, N, scale, stream);
-  return causal ? launch_fwd<128, true>(mq, mk, mv, o, lse, B, Hq, Hkv, N, scale, stream)
-                : launch_fwd<128, false>(mq, mk, mv, o, lse, B, Hq, Hkv, N, scale, stream);
+  return fwd_impl(q, k, v, o, lse, B, Hq, Hkv, N, N, d, scale, causal, -1, -1,
+                  static_cast<cudaStream_t>(stream_));
+}
+
+attn_status attn_fwd_masked(const void* q, const void* k, const void* v, void* o, float* lse,
+                            int B, int Hq, int Hkv, int Nq, int Nk, int d, float scale,
+                            int causal, int window_left, int window_right,
+                            attn_stream_t stream_) {
+  return fwd_impl(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, scale, causal, window_left,
+                  window_right, static_cast<cudaStream_t>(stream_));
 }
 
 size_t attn_bwd_workspace_size(int B, int Hq, int N, int d) {
@@ -396,78 +554,26 @@ attn_status attn_bwd(const void* q, const void* k, const void* v, const void* o,
                      const float* lse, const void* dO, void* dq, void* dk, void* dv,
                      void* workspace, size_t workspace_bytes, int B, int Hq, int Hkv, int N,
                      int d, float scale, int causal, attn_stream_t stream_) {
-  g_last_error[0] = '\0';
-  bool empty = false;
-  attn_status st = check_shape(B, Hq, Hkv, N, d, scale, &empty);
-  if (st != ATTN_OK) return st;
-  if (causal != 0 && causal != 1) return fail(ATTN_ERR_ARG, "causal must be 0 or 1");
-  if (empty) return ATTN_OK;
-  const void* ptrs[10] = {q, k, v, o, lse, dO, dq, dk, dv, workspace};
-  const char* names[10] = {"q", "k", "v", "o", "lse", "dO", "dq", "dk", "dv", "workspace"};
-  for (int i = 0; i < 10; ++i) {
-    if (ptrs[i] == nullptr) return fail(ATTN_ERR_ARG, "%s is null", names[i]);
-    if (!aligned16(ptrs[i])) return fail(ATTN_ERR_ARG, "%s is not 16-byte aligned", names[i]);
-  }
-  const size_t need = attn_bwd_workspace_size(B, Hq, N, d);
-  if (workspace_bytes < need)
-    return fail(ATTN_ERR_ARG, "workspace is %zu bytes, needs %zu", workspace_bytes, need);
-  st = ensure_init();
-  if (st != ATTN_OK) return st;
-  if ((st = check_ptrs(ptrs, names, 10)) != ATTN_OK) return st;
-  cudaStream_t stream = static_cast<cudaStream_t>(stream_);
-  CUtensorMap mq, mk, mv, mdo;
-  if ((st = make_map(&mq, q, d, N, B * Hq)) != ATTN_OK) return st;
-  if ((st = make_map(&mk, k, d, N, B * Hkv)) != ATTN_OK) return st;
-  if ((st = make_map(&mv, v, d, N, B * Hkv)) != ATTN_OK) return st;
-  if ((st = make_map(&mdo, dO, d, N, B * Hq)) != ATTN_OK) return st;
-  float* L = static_cast<float*>(workspace);
-  float* Dv = L + static_cast<size_t>(B) * Hq * attn::pad128(N);
-  BwdArgs a{mq, mk, mv, mdo, o, lse, dO, dq, dk, dv, L, Dv, B, Hq, Hkv, N, scale};
-  if (d == 64) return causal ? launch_bwd<64, true>(a, stream) : launch_bwd<64, false>(a, stream);
-  return causal ? launch_bwd<128, true>(a, stream) : launch_bwd<128, false>(a, stream);
+  return bwd_impl(q, k, v, o, lse, dO, dq, dk, dv, workspace, workspace_bytes, false, B, Hq, Hkv,
+                  N, N, d, scale, causal, -1, -1, static_cast<cudaStream_t>(stream_));
+}
+
+attn_status attn_bwd_masked(const void* q, const void* k, const void* v, const void* o,
+                            const float* lse, const void* dO, void* dq, void* dk, void* dv,
+                            void* workspace, size_t workspace_bytes, int B, int Hq, int Hkv,
+                            int Nq, int Nk, int d, float scale, int causal, int window_left,
+                            int window_right, attn_stream_t stream_) {
+  return bwd_impl(q, k, v, o, lse, dO, dq, dk, dv, workspace, workspace_bytes, false, B, Hq, Hkv,
+                  Nq, Nk, d, scale, causal, window_left, window_right,
+                  static_cast<cudaStream_t>(stream_));
 }
 
 attn_status attn_bwd_noalloc(const void* q, const void* k, const void* v, const void* o,
                              const float* lse, const void* dO, void* dq, void* dk, void* dv,
                              int B, int Hq, int Hkv, int N, int d, float scale, int causal,
                              attn_stream_t stream_) {
-  g_last_error[0] = '\0';
-  bool empty = false;
-  attn_status st = check_shape(B, Hq, Hkv, N, d, scale, &empty);
-  if (st != ATTN_OK) return st;
-  if (causal != 0 && causal != 1) return fail(ATTN_ERR_ARG, "causal must be 0 or 1");
-  if (empty) return ATTN_OK;
-  const void* ptrs[9] = {q, k, v, o, lse, dO, dq, dk, dv};
-  const char* names[9] = {"q", "k", "v", "o", "lse", "dO", "dq", "dk", "dv"};
-  for (int i = 0; i < 9; ++i) {
-    if (ptrs[i] == nullptr) return fail(ATTN_ERR_ARG, "%s is null", names[i]);
-    if (!aligned16(ptrs[i])) return fail(ATTN_ERR_ARG, "%s is not 16-byte aligned", names[i]);
-  }
-  const size_t need = attn_bwd_workspace_size(B, Hq, N, d);
-  if (need > kStaticScratchBytes)
-    return fail(ATTN_ERR_ARG,
-                "attn_bwd_noalloc: this shape needs %zu bytes of scratch, but the static area "
-                "holds %zu (B*Hq*ceil128(N) must be <= %zu); use attn_bwd with a workspace",
-                need, kStaticScratchBytes, kStaticScratchBytes / (2 * sizeof(float)));
-  st = ensure_init();
-  if (st != ATTN_OK) return st;
-  if ((st = check_ptrs(ptrs, names, 9)) != ATTN_OK) return st;
-  void* scratch = nullptr;
-  if ((st = static_scratch_ptr(&scratch)) != ATTN_OK) return st;
-  cudaStream_t stream = static_cast<cudaStream_t>(stream_);
-  CUtensorMap mq, mk, mv, mdo;
-  if ((st = make_map(&mq, q, d, N, B * Hq)) != ATTN_OK) return st;
-  if ((st = make_map(&mk, k, d, N, B * Hkv)) != ATTN_OK) return st;
-  if ((st = make_map(&mv, v, d, N, B * Hkv)) != ATTN_OK) return st;
-  if ((st = make_map(&mdo, dO, d, N, B * Hq)) != ATTN_OK) return st;
-  // The preprocess kernel writes every scratch row the other two kernels read,
-  // so nothing left over from an earlier call is ever used and no clearing
-  // is needed.
-  float* L = static_cast<float*>(scratch);
-  float* Dv = L + static_cast<size_t>(B) * Hq * attn::pad128(N);
-  BwdArgs a{mq, mk, mv, mdo, o, lse, dO, dq, dk, dv, L, Dv, B, Hq, Hkv, N, scale};
-  if (d == 64) return causal ? launch_bwd<64, true>(a, stream) : launch_bwd<64, false>(a, stream);
-  return causal ? launch_bwd<128, true>(a, stream) : launch_bwd<128, false>(a, stream);
+  return bwd_impl(q, k, v, o, lse, dO, dq, dk, dv, nullptr, 0, true, B, Hq, Hkv, N, N, d, scale,
+                  causal, -1, -1, static_cast<cudaStream_t>(stream_));
 }
 
 attn_status attn_selftest_wait_timeout(attn_stream_t stream_) {

@@ -34,6 +34,7 @@
 #pragma once
 
 #include "sm100.cuh"
+#include "visibility.cuh"
 
 namespace attn {
 
@@ -75,7 +76,9 @@ bwd_pre_kernel(const __nv_bfloat16* __restrict__ o, const __nv_bfloat16* __restr
   acc += __shfl_xor_sync(0xffffffffu, acc, 2);
   acc += __shfl_xor_sync(0xffffffffu, acc, 1);
   if (sub == 0) {
-    L[row] = (n < N) ? -lse[static_cast<size_t>(bh) * N + n] * kLog2e : -INFINITY;
+    const float l = (n < N) ? lse[static_cast<size_t>(bh) * N + n] : -INFINITY;
+    // A row that saw no key (lse = -inf) is treated like padding: P = 0.
+    L[row] = (l == -INFINITY) ? -INFINITY : -l * kLog2e;
     Dv[row] = (n < N) ? -acc : 0.f;
   }
 }
@@ -157,13 +160,13 @@ struct DkdvCfg {
   static constexpr int kThreads = 384;
 };
 
-template <int D, bool CAUSAL>
+template <int D, int MODE>
 __global__ void __launch_bounds__(384, 1)
 bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
                 const float* __restrict__ Lws, const float* __restrict__ Dws,
                 __nv_bfloat16* __restrict__ dk, __nv_bfloat16* __restrict__ dv, int Hq, int group,
-                int N, int Npad, float scale_log2, float scale) {
+                int Nq, int Nk, int Npad, float scale_log2, float scale, KeyWindow win) {
   using C = DkdvCfg<D>;
   constexpr int NS = C::kStages;
   extern __shared__ uint8_t smem_raw[];
@@ -187,14 +190,15 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   // 1-D grid, KV block fastest, then (batch, KV head): CTAs resident
   // together mostly share one head's Q/dO in L2. Low j has the most causal
   // work and launches first within its head.
-  const int nq = (N + 127) >> 7;
-  const int bh_kv = blockIdx.x / nq;
+  const int nkv = (Nk + 127) >> 7;
+  const int bh_kv = blockIdx.x / nkv;
   const int b = bh_kv / Hkv;
   const int hkv = bh_kv - b * Hkv;
-  const int j = blockIdx.x - bh_kv * nq;
-  const int i_start = CAUSAL ? j : 0;
-  const int per_head = nq - i_start;
-  const int n_steps = group * per_head;       // >= 1
+  const int j = blockIdx.x - bh_kv * nkv;
+  int i_start, i_end;                         // query blocks that see key tile j
+  q_block_range<MODE>(j, Nq, Nk, win, i_start, i_end);
+  const int per_head = max(0, i_end - i_start + 1);
+  const int n_steps = group * per_head;       // 0: no query sees these keys
 
   if (threadIdx.x == 0) {
     mbar_init(kv_full, 1);
@@ -233,11 +237,13 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_v);
       tma_prefetch_desc(&tm_do);
-      mbar_expect_tx(kv_full, 2 * C::kTile);
+      if (n_steps > 0) {
+        mbar_expect_tx(kv_full, 2 * C::kTile);
 #pragma unroll
-      for (int a = 0; a < D / 64; ++a) {
-        tma_load_3d(smem + C::kKOff + a * 16384, &tm_k, kv_full, a * 64, j * 128, bh_kv);
-        tma_load_3d(smem + C::kVOff + a * 16384, &tm_v, kv_full, a * 64, j * 128, bh_kv);
+        for (int a = 0; a < D / 64; ++a) {
+          tma_load_3d(smem + C::kKOff + a * 16384, &tm_k, kv_full, a * 64, j * 128, bh_kv);
+          tma_load_3d(smem + C::kVOff + a * 16384, &tm_v, kv_full, a * 64, j * 128, bh_kv);
+        }
       }
       int issued = 0;
       for (int s = 0; s < n_steps; ++s) {
@@ -257,7 +263,7 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         bulk_load(stage + 2 * C::kTile + 512, Dws + off, 512, &ld_full[st]);
         ++issued;
       }
-      mbar_wait_drain(kv_full, 0);
+      if (n_steps > 0) mbar_wait_drain(kv_full, 0);
       const int first = issued > NS ? issued - NS : 0;
       for (int s = first; s < issued; ++s) mbar_wait_drain(&ld_full[s % NS], (s / NS) & 1);
     }
@@ -283,7 +289,7 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
           mma_ts(acc, a_tmem + split_col(kk), sdesc_sw128(b + kk * 2048, 16384, 1024), kIdescAcc,
                  (accumulate || kk > 0) ? 1u : 0u);
       };
-      bool ok = mbar_wait(kv_full, 0, abort_flag, kSiteBKV) &&
+      bool ok = n_steps > 0 && mbar_wait(kv_full, 0, abort_flag, kSiteBKV) &&
                 mbar_wait(&ld_full[0], 0, abort_flag, kSiteBLoadFull);
       if (ok) {
         tc_fence_after();
@@ -317,8 +323,10 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         }
       }
       if (ok) tc_commit(acc_done);
-      tc_commit(mma_done);
-      mbar_wait_drain(mma_done, 0);
+      if (n_steps > 0) {                     // nothing to drain when nothing was issued
+        tc_commit(mma_done);
+        mbar_wait_drain(mma_done, 0);
+      }
     }
     __syncwarp();
   } else if (warp < 8) {
@@ -327,6 +335,8 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     const int quad = warp & 3;
     const int t = quad * 32 + lane;                   // key row within the block
     const int key = j * 128 + t;
+    // Query q sees this key iff key - off - wr <= q <= key - off + wl.
+    const int q_first = key - win.off - win.wr, q_last = key - win.off + win.wl;
     const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
     const uint32_t t_s = tmem + lane_base + 64 * h;          // S^T half; P^T into +0..32
     const uint32_t t_dp = tmem + lane_base + 128 + 64 * h;   // dP^T half; dS^T into +0..32
@@ -350,7 +360,14 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       tmem_ld32(t_s + 32, r1);
       tmem_ld_wait(r0);
       reg_fence(r1);
-      const bool diag = CAUSAL && (i == j);           // key t sees query c only if c >= t
+      // Masked steps: the causal diagonal, or (general mode) query blocks at
+      // an edge of the key tile's visibility band.
+      bool edge;
+      if (MODE == kMaskNone) edge = false;
+      else if (MODE == kMaskCausal) edge = i == j;
+      else edge = j * 128 < win.lo(min(i * 128 + 127, Nq - 1)) ||
+                  j * 128 + 127 > win.hi(i * 128);
+      const int c_lo = q_first - i * 128, c_hi = q_last - i * 128;   // keep columns [c_lo, c_hi]
       const float2 sc2 = make_float2(scale_log2, scale_log2);
       float pf[64];                                   // P in fp32 (for dS)
       uint32_t pw[32];                                // P as bf16 pairs (for the dV MMA)
@@ -362,9 +379,9 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
           const float2 x = ffma2(make_float2(u2f(r[2 * e]), u2f(r[2 * e + 1])), sc2, nl);
           float p0 = fast_exp2(x.x);
           float p1 = fast_exp2(x.y);
-          if (diag) {
-            if (c < t) p0 = 0.f;
-            if (c + 1 < t) p1 = 0.f;
+          if (edge) {
+            if (c < c_lo || c > c_hi) p0 = 0.f;
+            if (c + 1 < c_lo || c + 1 > c_hi) p1 = 0.f;
           }
           pf[c0 + 2 * e] = p0;
           pf[c0 + 2 * e + 1] = p1;
@@ -397,15 +414,22 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       tc_fence_before();
       mbar_arrive(ds_full);
     }
-    if (ok) ok = mbar_wait(acc_done, 0, abort_flag, kSiteBAcc);
+    if (ok && n_steps > 0) ok = mbar_wait(acc_done, 0, abort_flag, kSiteBAcc);
     if (ok) {
-      tc_fence_after();
-      const bool valid = key < N;
-      const size_t row_off = (static_cast<size_t>(bh_kv) * N + (valid ? key : 0)) * D;
-      if (h == 0)
-        store_acc_row<D>(tmem + lane_base + 256, dv + row_off, 1.0f, valid);
-      else
-        store_acc_row<D>(tmem + lane_base + 384, dk + row_off, scale, valid);
+      const bool valid = key < Nk;
+      const size_t row_off = (static_cast<size_t>(bh_kv) * Nk + (valid ? key : 0)) * D;
+      if (n_steps > 0) {
+        tc_fence_after();
+        if (h == 0)
+          store_acc_row<D>(tmem + lane_base + 256, dv + row_off, 1.0f, valid);
+        else
+          store_acc_row<D>(tmem + lane_base + 384, dk + row_off, scale, valid);
+      } else if (valid) {
+        // No query sees these keys: their gradients are zero.
+        uint4* dst = reinterpret_cast<uint4*>((h == 0 ? dv : dk) + row_off);
+#pragma unroll
+        for (int c = 0; c < D / 8; ++c) dst[c] = make_uint4(0u, 0u, 0u, 0u);
+      }
     }
   }
 
@@ -434,13 +458,13 @@ struct DqCfg {
   static constexpr int kThreads = 384;
 };
 
-template <int D, bool CAUSAL>
+template <int D, int MODE>
 __global__ void __launch_bounds__(384, 1)
 bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
               const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
               const float* __restrict__ Lws, const float* __restrict__ Dws,
-              __nv_bfloat16* __restrict__ dq, int Hq, int group, int N, int Npad, float scale_log2,
-              float scale) {
+              __nv_bfloat16* __restrict__ dq, int Hq, int group, int Nq, int Nk, int Npad,
+              float scale_log2, float scale, KeyWindow win) {
   using C = DqCfg<D>;
   constexpr int NS = C::kStages;
   extern __shared__ uint8_t smem_raw[];
@@ -462,13 +486,16 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
   const int warp = warp_id(), lane = lane_id();
   // 1-D grid, query block fastest (heaviest causal block first), then
   // (batch, query head): CTAs resident together mostly share one head's K/V.
-  const int nkv = (N + 127) >> 7;
-  const int bh = blockIdx.x / nkv;
+  const int nqb = (Nq + 127) >> 7;
+  const int nkv = (Nk + 127) >> 7;
+  const int bh = blockIdx.x / nqb;
   const int b = bh / Hq;
   const int hq = bh - b * Hq;
   const int bh_kv = b * (Hq / group) + hq / group;
-  const int i = nkv - 1 - (blockIdx.x - bh * nkv);
-  const int n = CAUSAL ? min(i + 1, nkv) : nkv;
+  const int i = nqb - 1 - (blockIdx.x - bh * nqb);
+  int j_lo, j_hi;                            // key tiles this query block sees
+  kv_tile_range<MODE>(i * 128, min(i * 128 + 127, Nq - 1), Nk, win, j_lo, j_hi);
+  const int n = max(0, j_hi - j_lo + 1);
 
   if (threadIdx.x == 0) {
     mbar_init(qd_full, 1);
@@ -501,11 +528,13 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_v);
       tma_prefetch_desc(&tm_do);
-      mbar_expect_tx(qd_full, 2 * C::kTile);
+      if (n > 0) {
+        mbar_expect_tx(qd_full, 2 * C::kTile);
 #pragma unroll
-      for (int a = 0; a < D / 64; ++a) {
-        tma_load_3d(smem + C::kQOff + a * 16384, &tm_q, qd_full, a * 64, i * 128, bh);
-        tma_load_3d(smem + C::kDOOff + a * 16384, &tm_do, qd_full, a * 64, i * 128, bh);
+        for (int a = 0; a < D / 64; ++a) {
+          tma_load_3d(smem + C::kQOff + a * 16384, &tm_q, qd_full, a * 64, i * 128, bh);
+          tma_load_3d(smem + C::kDOOff + a * 16384, &tm_do, qd_full, a * 64, i * 128, bh);
+        }
       }
       uint32_t issued = 0;
       bool ok = true;
@@ -520,11 +549,11 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
 #pragma unroll
           for (int a = 0; a < D / 64; ++a)
             tma_load_3d(smem + C::kKVOff + s * C::kTile + a * 16384, w ? &tm_v : &tm_k, &kv_full[s],
-                        a * 64, jj * 128, bh_kv);
+                        a * 64, (j_lo + jj) * 128, bh_kv);
           ++issued;
         }
       }
-      mbar_wait_drain(qd_full, 0);
+      if (n > 0) mbar_wait_drain(qd_full, 0);
       const uint32_t first = issued > (uint32_t)NS ? issued - NS : 0u;
       for (uint32_t x = first; x < issued; ++x) mbar_wait_drain(&kv_full[x % NS], (x / NS) & 1u);
     }
@@ -545,7 +574,7 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                  kk > 0 ? 1u : 0u);
         }
       };
-      bool ok = mbar_wait(qd_full, 0, abort_flag, kSiteBLoadFull) && kv_wait(0);
+      bool ok = n > 0 && mbar_wait(qd_full, 0, abort_flag, kSiteBLoadFull) && kv_wait(0);
       if (ok) {
         tc_fence_after();
         mma_tile_kk(tmem + 0, sbase + C::kQOff, slot(0));        // S(0) = Q K_0^T
@@ -586,8 +615,10 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         }
       }
       if (ok) tc_commit(acc_done);
-      tc_commit(mma_done);
-      mbar_wait_drain(mma_done, 0);
+      if (n > 0) {                           // nothing to drain when nothing was issued
+        tc_commit(mma_done);
+        mbar_wait_drain(mma_done, 0);
+      }
     }
     __syncwarp();
   } else if (warp < 8) {
@@ -596,6 +627,11 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     const int quad = warp & 3;
     const int t = quad * 32 + lane;                  // query row within the block
     const int row = i * 128 + t;
+    const int r_first = i * 128, r_last = min(i * 128 + 127, Nq - 1);
+    // Visible keys of this row: [k_lo, k_hi].
+    const int k_lo = (MODE == kMaskGeneral) ? max(0, win.lo(row)) : 0;
+    const int k_hi = (MODE == kMaskGeneral) ? min(Nk - 1, win.hi(row))
+                                            : ((MODE == kMaskCausal) ? min(row, Nk - 1) : Nk - 1);
     const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
     const uint32_t t_s = tmem + lane_base + 64 * h;
     const uint32_t t_dp = tmem + lane_base + 128 + 64 * h;   // dP half; dS into +0..32
@@ -614,11 +650,15 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
       reg_fence(r1);
       tc_fence_before();
       mbar_arrive(s_free);
-      const bool diag = CAUSAL && (jj == i);          // query t sees key c only if c <= t
-      // Keys past N (zero rows from the TMA fill) get P = 0 explicitly, so an
-      // extreme lse can never turn 0 * exp2(-lse) into a NaN.
-      const int klim = N - jj * 128;
-      const bool ragged_tile = (jj == nkv - 1) && (N & 127) != 0;
+      const int kb = (j_lo + jj) * 128;
+      // Masked tiles: those crossing an edge of some row's visible keys,
+      // including the ragged last tile (keys past Nk are zero rows from the
+      // TMA fill; P = 0 there keeps an extreme lse from making 0 * inf).
+      bool edge;
+      if (MODE == kMaskNone) edge = kb + 127 >= Nk;
+      else if (MODE == kMaskCausal) edge = kb + 127 > min(r_first, Nk - 1) || kb + 127 >= Nk;
+      else edge = kb < (r_last >= 0 ? win.lo(r_last) : 0) || kb + 127 > min(Nk - 1, win.hi(r_first));
+      const int c_lo = k_lo - kb, c_hi = k_hi - kb;   // keep columns [c_lo, c_hi]
       const float2 sc2 = make_float2(scale_log2, scale_log2);
       const float2 nl2 = make_float2(nLr, nLr);
       float pf[64];                                   // P in fp32
@@ -629,13 +669,9 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
           const float2 x = ffma2(make_float2(u2f(r[2 * e]), u2f(r[2 * e + 1])), sc2, nl2);
           float p0 = fast_exp2(x.x);
           float p1 = fast_exp2(x.y);
-          if (diag) {
-            if (c > t) p0 = 0.f;
-            if (c + 1 > t) p1 = 0.f;
-          }
-          if (ragged_tile) {
-            if (c >= klim) p0 = 0.f;
-            if (c + 1 >= klim) p1 = 0.f;
+          if (edge) {
+            if (c < c_lo || c > c_hi) p0 = 0.f;
+            if (c + 1 < c_lo || c + 1 > c_hi) p1 = 0.f;
           }
           pf[c0 + 2 * e] = p0;
           pf[c0 + 2 * e + 1] = p1;
@@ -662,15 +698,22 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
       tc_fence_before();
       mbar_arrive(ds_full);
     }
-    if (ok) ok = mbar_wait(acc_done, 0, abort_flag, kSiteBAcc);
+    if (ok && n > 0) ok = mbar_wait(acc_done, 0, abort_flag, kSiteBAcc);
     if (ok) {
-      tc_fence_after();
-      const bool valid = row < N;
-      __nv_bfloat16* dst = dq + (static_cast<size_t>(bh) * N + (valid ? row : 0)) * D;
-      if (h == 0)
-        store_acc_row<D, 0, D / 64>(tmem + lane_base + 256, dst, scale, valid);
-      else
-        store_acc_row<D, D / 64, D / 32>(tmem + lane_base + 256, dst, scale, valid);
+      const bool valid = row < Nq;
+      __nv_bfloat16* dst = dq + (static_cast<size_t>(bh) * Nq + (valid ? row : 0)) * D;
+      if (n > 0) {
+        tc_fence_after();
+        if (h == 0)
+          store_acc_row<D, 0, D / 64>(tmem + lane_base + 256, dst, scale, valid);
+        else
+          store_acc_row<D, D / 64, D / 32>(tmem + lane_base + 256, dst, scale, valid);
+      } else if (valid) {
+        // This query block sees no key: its gradient is zero.
+        uint4* p = reinterpret_cast<uint4*>(dst) + h * (D / 16);
+#pragma unroll
+        for (int c = 0; c < D / 16; ++c) p[c] = make_uint4(0u, 0u, 0u, 0u);
+      }
     }
   }
 

@@ -38,6 +38,7 @@
 #pragma once
 
 #include "sm100.cuh"
+#include "visibility.cuh"
 
 namespace attn {
 
@@ -74,11 +75,12 @@ constexpr int kFwdRegsSoftmax = 216;
 constexpr int kFwdRegsSmall = 72;
 static_assert(2 * kFwdRegsSoftmax + kFwdRegsSmall <= 3 * kFwdRegsLaunch, "register split");
 
-template <int D, bool CAUSAL>
+template <int D, int MODE>
 __global__ void __launch_bounds__(384, 1)
 fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
            const __grid_constant__ CUtensorMap tm_v, __nv_bfloat16* __restrict__ out,
-           float* __restrict__ lse_out, int Hq, int group, int N, float scale_log2) {
+           float* __restrict__ lse_out, int Hq, int group, int Nq, int Nk, float scale_log2,
+           KeyWindow win) {
   using C = FwdCfg<D>;
   constexpr int NS = C::kStages;
   extern __shared__ uint8_t smem_raw[];
@@ -101,22 +103,33 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
   // 1-D grid, (batch, query head) fastest, then 256-row query block from the
   // last (heaviest when causal) to the first: every head's heaviest block is
   // dispatched before any lighter one, which keeps the causal tail short.
-  const int nmb = (N + 255) >> 8;
+  const int nmb = (Nq + 255) >> 8;
   const int BH = gridDim.x / nmb;
   const int bh = blockIdx.x % BH;                  // b * Hq + hq
   const int b = bh / Hq;
   const int hq = bh - b * Hq;
   const int bh_kv = b * (Hq / group) + hq / group; // GQA: contiguous head groups
   const int mb = nmb - 1 - static_cast<int>(blockIdx.x / BH);
-  const int nkv = (N + 127) >> 7;
+  const int nkv = (Nk + 127) >> 7;
 
-  int n_t[2];
+  // Per query tile t: KV tiles [lo_t[t], hi_t[t]] (n_t[t] of them). A tile whose
+  // rows exist but see no key has n_t = 0 and writes O = 0, lse = -inf. The
+  // CTA streams KV tiles jb..je, the union of its tiles' ranges.
+  int lo_t[2], hi_t[2], n_t[2];
 #pragma unroll
   for (int t = 0; t < 2; ++t) {
     const int r0 = mb * 256 + t * 128;
-    n_t[t] = (r0 >= N) ? 0 : (CAUSAL ? min(nkv, (r0 >> 7) + 1) : nkv);
+    if (r0 >= Nq) {
+      lo_t[t] = 0;
+      hi_t[t] = -1;
+    } else {
+      kv_tile_range<MODE>(r0, min(r0 + 127, Nq - 1), Nk, win, lo_t[t], hi_t[t]);
+    }
+    n_t[t] = max(0, hi_t[t] - lo_t[t] + 1);
   }
-  const int n_max = max(n_t[0], n_t[1]);
+  const int jb = (n_t[0] > 0) ? lo_t[0] : lo_t[1];
+  const int je = (n_t[1] > 0) ? hi_t[1] : hi_t[0];
+  const int n_span = (n_t[0] > 0 || n_t[1] > 0) ? je - jb + 1 : 0;
 
   if (threadIdx.x == 0) {
     mbar_init(&q_full[0], 1);
@@ -162,7 +175,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
       }
       uint32_t issued = 0;
       bool ok = true;
-      for (int j = 0; j < n_max && ok; ++j) {
+      for (int j = jb; j < jb + n_span && ok; ++j) {
         for (int w = 0; w < 2; ++w) {
           const uint32_t s = issued % NS;
           const uint32_t round = issued / NS;
@@ -213,47 +226,64 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
 #pragma unroll
       for (int t = 0; t < 2; ++t)
         if (ok && n_t[t] > 0) ok = mbar_wait(&q_full[t], 0, abort_flag, kSiteQFull);
-      if (ok) ok = kv_wait(0);
-      if (ok) {
+      // Ring positions: K_j at 2 (j - jb), V_j at 2 (j - jb) + 1.
+      if (ok && n_span > 0) ok = kv_wait(0);
+      if (ok && n_span > 0) {
         tc_fence_after();
 #pragma unroll
         for (int t = 0; t < 2; ++t)
-          if (n_t[t] > 0) {
+          if (n_t[t] > 0 && lo_t[t] == jb) {
             issue_qk(t, 0);
             tc_commit(&s_full[t]);
           }
         tc_commit(&kv_empty[0]);
       }
-      for (int j = 0; ok && j < n_max; ++j) {
-        const uint32_t iv = 2 * j + 1, ik = 2 * j + 2;
+      for (int j = jb; ok && j < jb + n_span; ++j) {
+        const uint32_t iv = 2 * (j - jb) + 1, ik = 2 * (j - jb) + 2;
         if (!kv_wait(iv)) { ok = false; break; }
         tc_fence_after();
         bool k_ready = false;
+        auto need_k_next = [&]() {
+          if (!k_ready) {
+            if (!kv_wait(ik)) return false;
+            tc_fence_after();
+            k_ready = true;
+          }
+          return true;
+        };
 #pragma unroll
         for (int t = 0; t < 2; ++t) {
-          if (j >= n_t[t]) continue;
-          if (!mbar_wait(&p_full[t], j & 1, abort_flag, kSitePFull)) { ok = false; break; }
-          tc_fence_after();
-          issue_pv(t, iv % NS, j > 0);
-          if (j == n_t[t] - 1) {
-            tc_commit(&o_full[t]);
-          } else {
-            if (!k_ready) {
-              if (!kv_wait(ik)) { ok = false; break; }
-              tc_fence_after();
-              k_ready = true;
+          if (n_t[t] == 0) continue;
+          if (j >= lo_t[t] && j <= hi_t[t]) {
+            if (!mbar_wait(&p_full[t], (j - lo_t[t]) & 1, abort_flag, kSitePFull)) { ok = false; break; }
+            tc_fence_after();
+            issue_pv(t, iv % NS, j > lo_t[t]);
+            if (j == hi_t[t]) {
+              tc_commit(&o_full[t]);
+            } else {
+              if (!need_k_next()) { ok = false; break; }
+              issue_qk(t, ik % NS);
+              tc_commit(&s_full[t]);
             }
+          } else if (lo_t[t] == j + 1) {
+            // This tile's first key tile is the next one.
+            if (!need_k_next()) { ok = false; break; }
             issue_qk(t, ik % NS);
             tc_commit(&s_full[t]);
           }
         }
+        // K_{j+1} feeds some tile whenever j + 1 is in the span (the two tiles'
+        // ranges overlap or touch); release its slot even if no tile used it.
+        if (ok && j + 1 < jb + n_span && !need_k_next()) ok = false;
         if (!ok) break;
         tc_commit(&kv_empty[iv % NS]);
         if (k_ready) tc_commit(&kv_empty[ik % NS]);
       }
       // Let this thread's MMAs finish before TMEM can be released.
-      tc_commit(mma_done);
-      mbar_wait_drain(mma_done, 0);
+      if (n_span > 0) {                       // nothing to drain when no tile was issued
+        tc_commit(mma_done);
+        mbar_wait_drain(mma_done, 0);
+      }
     }
     __syncwarp();
   } else {
@@ -267,15 +297,22 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
     const uint32_t t_p = t_s + 64;
     const uint32_t t_o = tmem + lane_base + 256 + t * 128;
     const int n = n_t[t];
-    const bool mask_last = CAUSAL || (N & 127) != 0;
-    const int visible_end = CAUSAL ? min(row + 1, N) : N;   // keys [0, visible_end) are visible
+    const int r_first = mb * 256 + t * 128;                  // first and last row of this tile
+    const int r_last = min(r_first + 127, Nq - 1);
+    // Visible keys of this row: [k_lo, k_hi] (k_hi < k_lo: none).
+    const int k_lo = (MODE == kMaskGeneral) ? max(0, win.lo(row)) : 0;
+    const int k_hi = (MODE == kMaskGeneral) ? min(Nk - 1, win.hi(row))
+                                            : ((MODE == kMaskCausal) ? min(row, Nk - 1) : Nk - 1);
+    const bool ragged = (Nk & 127) != 0;
 
     float m_run = -INFINITY;   // running max, log2 units (scaled logits * log2 e)
     float l_run = 0.f;         // running sum of 2^(t - m_run), unrounded (for lse)
     float l_mma = 0.f;         // running sum of the bf16-rounded P fed to the MMA (for O)
     bool ok = n > 0;
-    for (int j = 0; ok && j < n; ++j) {
-      if (!mbar_wait(&s_full[t], j & 1, abort_flag, kSiteSFull)) { ok = false; break; }
+    for (int jj = 0; ok && jj < n; ++jj) {
+      const int j = lo_t[t] + jj;                            // key tile
+      const int kb = j * 128;
+      if (!mbar_wait(&s_full[t], jj & 1, abort_flag, kSiteSFull)) { ok = false; break; }
       tc_fence_after();
       uint32_t r0[32], r1[32], r2[32], r3[32];
       tmem_ld32(t_s + 0, r0);
@@ -287,15 +324,20 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
       reg_fence(r2);
       reg_fence(r3);
 
-      if (mask_last && j == n - 1) {
-        const int lim = visible_end - j * 128;   // columns [lim, 128) are masked
+      // Only tiles that straddle an edge of some row's visible range are masked.
+      bool edge;
+      if (MODE == kMaskNone) edge = ragged && j == nkv - 1;
+      else if (MODE == kMaskCausal) edge = jj == n - 1;
+      else edge = kb < win.lo(r_last) || kb + 127 > min(Nk - 1, win.hi(r_first));
+      if (edge) {
+        const int c_lo = k_lo - kb, c_hi = k_hi - kb;     // keep columns [c_lo, c_hi]
         const uint32_t ninf = f2u(-INFINITY);
 #pragma unroll
         for (int e = 0; e < 32; ++e) {
-          if (e >= lim) r0[e] = ninf;
-          if (32 + e >= lim) r1[e] = ninf;
-          if (64 + e >= lim) r2[e] = ninf;
-          if (96 + e >= lim) r3[e] = ninf;
+          if (e < c_lo || e > c_hi) r0[e] = ninf;
+          if (32 + e < c_lo || 32 + e > c_hi) r1[e] = ninf;
+          if (64 + e < c_lo || 64 + e > c_hi) r2[e] = ninf;
+          if (96 + e < c_lo || 96 + e > c_hi) r3[e] = ninf;
         }
       }
       float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
@@ -310,7 +352,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
       const float m_new = fmaxf(m_run, m_tile);
       // Lazy rescale: keep the stale max unless the new one is more than 2^8 larger.
       const bool need = m_new > m_run + 8.0f;
-      if (j > 0 && __any_sync(0xffffffffu, need)) {
+      if (jj > 0 && __any_sync(0xffffffffu, need)) {
         const float f = need ? fast_exp2(m_run - m_new) : 1.0f;
 #pragma unroll
         for (int c = 0; c < D / 32; ++c) {
@@ -329,7 +371,9 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
         m_run = m_new;
       }
       const float2 sc2 = make_float2(scale_log2, scale_log2);
-      const float2 nm2 = make_float2(-m_run, -m_run);
+      // A row with no visible key so far keeps m_run = -inf; its p are all 0.
+      const float neg_m = (m_run == -INFINITY) ? 0.0f : -m_run;
+      const float2 nm2 = make_float2(neg_m, neg_m);
       float2 ex0 = make_float2(0.f, 0.f), ex1 = make_float2(0.f, 0.f);
       float q0 = 0.f, q1 = 0.f, q2 = 0.f, q3 = 0.f;
       // Exponentiate 32 columns at a time and store them as 16 packed bf16
@@ -369,20 +413,28 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
       mbar_arrive(&p_full[t]);
     }
 
+    // Epilogue. A row that saw no key (l = 0) gets O = 0 and lse = -inf.
+    const bool present = r_first < Nq;
     if (ok) ok = mbar_wait(&o_full[t], 0, abort_flag, kSiteOFull);
-    if (ok) {
-      tc_fence_after();
-      const float inv_l = 1.0f / l_mma;
-      __nv_bfloat16* orow = out + (static_cast<size_t>(bh) * N + row) * D;
+    if (ok || (present && n == 0)) {
+      const bool has_o = n > 0;
+      if (has_o) tc_fence_after();
+      const float inv_l = (l_mma > 0.f) ? 1.0f / l_mma : 0.f;
+      __nv_bfloat16* orow = out + (static_cast<size_t>(bh) * Nq + (row < Nq ? row : 0)) * D;
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
         uint32_t o[32];
-        tmem_ld32(t_o + c * 32, o);
-        tmem_ld_wait(o);
+        if (has_o) {
+          tmem_ld32(t_o + c * 32, o);
+          tmem_ld_wait(o);
+        } else {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) o[e] = 0u;
+        }
         uint32_t pk[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e) pk[e] = pack_bf16x2(u2f(o[2 * e]) * inv_l, u2f(o[2 * e + 1]) * inv_l);
-        if (row < N) {
+        if (row < Nq) {
           uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
           dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
           dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
@@ -390,8 +442,9 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
           dst[3] = make_uint4(pk[12], pk[13], pk[14], pk[15]);
         }
       }
-      if (row < N)
-        lse_out[static_cast<size_t>(bh) * N + row] = (m_run + __log2f(l_run)) * 0.69314718055994531f;
+      if (row < Nq)
+        lse_out[static_cast<size_t>(bh) * Nq + row] =
+            (l_run > 0.f) ? (m_run + __log2f(l_run)) * 0.69314718055994531f : -INFINITY;
     }
   }
 

@@ -8,11 +8,14 @@
  *
  *     O = softmax(Q @ K^T * softmax_scale) @ V
  *
- * `causal` masks key j for query i when j > i. The bottom-right alignment
- * (same page, section "Von 2.0 bis 2.7", release 2.1) is the same thing here,
- * because queries and keys always have the same length N. K and V may have
- * fewer heads than Q when Hq is divisible by Hkv (MQA/GQA, same interface
- * section). Query head h reads KV head h / (Hq / Hkv).
+ * `causal` masks key j for query i when j > i. In attn_fwd/attn_bwd queries
+ * and keys have the same length N. attn_fwd_masked/attn_bwd_masked take
+ * Nq != Nk and a sliding window. There the causal mask is aligned to the
+ * bottom-right corner (same page, section "Von 2.0 bis 2.7", release 2.1),
+ * and the window of release 2.3 (`window_size` in the interface section)
+ * applies. K and V may have fewer heads than Q when Hq is divisible by Hkv
+ * (MQA/GQA, same interface section). Query head h reads KV head
+ * h / (Hq / Hkv).
  *
  * The method is exact, not an approximation (tokenwerk.de "FlashAttention",
  * section "Was FlashAttention veraendert"). Results differ from a float64
@@ -134,6 +137,40 @@ attn_status attn_bwd_noalloc(const void* q, const void* k, const void* v, const 
                              attn_stream_t stream);
 
 /*
+ * attn_fwd_masked: attn_fwd with Nq queries, Nk keys and a sliding window.
+ *   q, o [B, Hq, Nq, d] bf16; k, v [B, Hkv, Nk, d] bf16; lse [B, Hq, Nq] f32.
+ *   With off = Nk - Nq, query row i sees key j (0 <= j < Nk) iff
+ *       i + off - window_left <= j <= i + off + window_right,
+ *   and, with causal = 1, also j <= i + off (so causal caps window_right at
+ *   0). A negative window side is unbounded. window_left = window_right = -1
+ *   and Nq == Nk is exactly attn_fwd.
+ *   A query row that sees no key (Nq > Nk with causal, or a window that
+ *   falls outside the keys) gets o = 0 and lse = -inf. Nk == 0 with Nq > 0
+ *   is such a case for every row. Nq == 0 or B == 0 writes nothing.
+ * Errors as in attn_fwd.
+ */
+attn_status attn_fwd_masked(const void* q, const void* k, const void* v, void* o, float* lse,
+                            int B, int Hq, int Hkv, int Nq, int Nk, int d, float scale,
+                            int causal, int window_left, int window_right,
+                            attn_stream_t stream);
+
+/*
+ * attn_bwd_masked: backward of attn_fwd_masked, with the same Nq, Nk,
+ * causal and window arguments.
+ *   dO, dq [B, Hq, Nq, d]; dk, dv [B, Hkv, Nk, d]; lse as attn_fwd_masked
+ *   wrote it. The workspace needs attn_bwd_workspace_size(B, Hq, Nq, d)
+ *   bytes. A query row that sees no key gets dq = 0. A key that no query
+ *   sees gets dk = dv = 0. With Nk == 0 only dq (zeros) is written; with
+ *   Nq == 0 only dk and dv (zeros).
+ * Errors as in attn_bwd.
+ */
+attn_status attn_bwd_masked(const void* q, const void* k, const void* v, const void* o,
+                            const float* lse, const void* dO, void* dq, void* dk, void* dv,
+                            void* workspace, size_t workspace_bytes, int B, int Hq, int Hkv,
+                            int Nq, int Nk, int d, float scale, int causal, int window_left,
+                            int window_right, attn_stream_t stream);
+
+/*
  * Synchronises `stream`, then reads and clears the device status word.
  * Returns ATTN_ERR_TIMEOUT if a kernel gave up on a wait since the last
  * check, ATTN_ERR_CUDA on a CUDA error, and ATTN_OK otherwise.
@@ -169,7 +206,7 @@ void attn_profile_enable(int on);
 void attn_profile_reset(void);
 attn_status attn_profile_read(int kernel, const char** name, int* launches, double* total_ms);
 
-/* ABI version of this header: major * 100 + minor. */
+/* ABI version of this header: major * 100 + minor (1.01: the masked calls). */
 int attn_abi_version(void);
 
 #ifdef __cplusplus

@@ -37,7 +37,7 @@ def test_library_exports_every_declared_symbol(lib):
     for name in declared_functions():
         assert hasattr(lib, name), name
     assert set(declared_functions()) <= set(ea.SIGNATURES)
-    assert lib.attn_abi_version() == 100
+    assert lib.attn_abi_version() == 101
 
 
 FAKE = 1 << 20          # aligned, non-null, but not device memory
@@ -117,3 +117,73 @@ def test_binding_rejects_cpu_tensors():
     q = torch.zeros(1, 1, 128, 64, dtype=torch.bfloat16)
     with pytest.raises(ValueError, match="CUDA"):
         ea.attn_fwd(q, q, q, o=q.clone(), lse=torch.zeros(1, 1, 128), causal=False)
+
+
+def fwd_masked(lib, q=FAKE, k=FAKE, v=FAKE, o=FAKE, lse=FAKE, B=1, Hq=2, Hkv=1, Nq=128, Nk=256,
+               d=64, scale=0.125, causal=0, wl=-1, wr=-1):
+    return lib.attn_fwd_masked(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, scale, causal, wl, wr, None)
+
+
+def bwd_masked(lib, ws=FAKE, ws_bytes=1 << 30, B=1, Hq=2, Hkv=1, Nq=128, Nk=256, d=64,
+               scale=0.125, causal=0, wl=-1, wr=-1, **ptrs):
+    p = {n: FAKE for n in ("q", "k", "v", "o", "lse", "dO", "dq", "dk", "dv")}
+    p.update(ptrs)
+    return lib.attn_bwd_masked(p["q"], p["k"], p["v"], p["o"], p["lse"], p["dO"], p["dq"],
+                               p["dk"], p["dv"], ws, ws_bytes, B, Hq, Hkv, Nq, Nk, d, scale,
+                               causal, wl, wr, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(Nq=-1), ea.ATTN_ERR_ARG),
+    (dict(Nk=-1), ea.ATTN_ERR_ARG),
+    (dict(Nk=(1 << 24) + 1), ea.ATTN_ERR_ARG),
+    (dict(causal=3), ea.ATTN_ERR_ARG),
+    (dict(Hq=3, Hkv=2), ea.ATTN_ERR_ARG),
+    (dict(d=80), ea.ATTN_ERR_UNSUPPORTED),
+    (dict(q=None), ea.ATTN_ERR_ARG),
+    (dict(v=FAKE + 2), ea.ATTN_ERR_ARG),
+    (dict(o=None, Nk=0), ea.ATTN_ERR_ARG),        # Nk == 0 still writes o and lse
+])
+def test_fwd_masked_argument_errors(lib, kw, code):
+    assert fwd_masked(lib, **kw) == code
+    assert lib.attn_get_last_error().decode() != ""
+
+
+def test_masked_empty_problems(lib):
+    # No query rows: nothing is written, so no pointer is needed.
+    assert fwd_masked(lib, q=None, k=None, v=None, o=None, lse=None, Nq=0) == ea.ATTN_OK
+    assert fwd_masked(lib, B=0) == ea.ATTN_OK
+    assert bwd_masked(lib, B=0) == ea.ATTN_OK
+    assert bwd_masked(lib, Nq=0, Nk=0, q=None, k=None, v=None, o=None, lse=None, dO=None,
+                      dq=None, dk=None, dv=None, ws=None) == ea.ATTN_OK
+
+
+def test_masked_no_keys_needs_no_key_pointers(lib):
+    """Nk == 0 with rows to write: k and v are not read, so null is accepted;
+    without a device the call then fails as a CUDA error, not an argument one."""
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    assert fwd_masked(lib, k=None, v=None, Nk=0) == ea.ATTN_ERR_CUDA
+    assert bwd_masked(lib, Nk=0, k=None, v=None, dk=None, dv=None, o=None, lse=None, dO=None,
+                      ws=None, ws_bytes=0) == ea.ATTN_ERR_CUDA
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(Nq=-3), ea.ATTN_ERR_ARG),
+    (dict(dk=None), ea.ATTN_ERR_ARG),
+    (dict(ws=None), ea.ATTN_ERR_ARG),
+    (dict(ws_bytes=2 * 2 * 128 * 4 - 4), ea.ATTN_ERR_ARG),   # workspace sized by Nq
+    (dict(causal=-1), ea.ATTN_ERR_ARG),
+])
+def test_bwd_masked_argument_errors(lib, kw, code):
+    assert bwd_masked(lib, **kw) == code
+
+
+def test_bwd_masked_workspace_is_sized_by_queries(lib):
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    need = lib.attn_bwd_workspace_size(1, 2, 128, 64)
+    # Exactly the Nq-sized workspace passes the argument checks (then: no device).
+    assert bwd_masked(lib, Nq=128, Nk=4096, ws_bytes=need) == ea.ATTN_ERR_CUDA

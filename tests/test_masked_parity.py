@@ -1,0 +1,239 @@
+"""GPU parity of the masked calls (attn_fwd_masked / attn_bwd_masked): query
+and key lengths that differ, with the causal mask aligned to the bottom-right
+corner (hysenlabs.com "FlashAttention: exakte Attention-Kernel fuer CUDA und
+ROCm", section "Von 2.0 bis 2.7", release 2.1), and sliding windows (release
+2.3, `window_size` in the interface section). The float64 oracle is the
+reference on the same seeded bf16 inputs.
+
+Rows that see no key must give O = 0 and lse = -inf exactly (the oracle's
+reading of an empty softmax), and their dQ = 0. Keys that no query sees get
+dK = dV = 0. Elsewhere the tolerances are those of the unmasked calls:
+|O - O_ref| <= 1e-2, |lse - lse_ref| <= 1e-3, and for each gradient
+max|got - ref| <= 2e-2 * max|ref| (absolute floor 1e-5)."""
+import numpy as np
+import pytest
+import torch
+
+import exact_attention_105_b200 as ea
+import oracle
+import workloads
+from tests.gpu_helpers import GRAD_REL_TOL, LSE_TOL, O_TOL, max_err, to_dev
+
+pytestmark = pytest.mark.gpu
+
+ZERO_REF_FLOOR = 1e-5
+
+
+def assert_masked_fwd_close(o, lse, o_ref, lse_ref, label):
+    o = o.float().cpu().numpy()
+    lse = lse.float().cpu().numpy()
+    assert np.all(np.isfinite(o)), f"{label}: non-finite O"
+    empty = np.isneginf(lse_ref)
+    assert np.array_equal(np.isneginf(lse), empty), \
+        f"{label}: rows with lse = -inf differ ({int(np.isneginf(lse).sum())} vs {int(empty.sum())})"
+    assert not np.any(np.isnan(lse)), f"{label}: NaN lse"
+    assert np.all(o[empty] == 0.0), f"{label}: O of a row with no visible key is not 0"
+    eo, io = max_err(o, o_ref)
+    assert eo <= O_TOL, f"{label}: max|O-O_ref| = {eo:.3e} at {io}"
+    if (~empty).any():
+        el, il = max_err(lse[~empty], lse_ref[~empty])
+        assert el <= LSE_TOL, f"{label}: max|lse-lse_ref| = {el:.3e}"
+    return eo
+
+
+def assert_masked_grads_close(got, refs, label, causal, window):
+    """Tolerance check, plus exact zeros where the mask alone makes a gradient
+    zero: dQ of query rows that see no key, dK/dV of keys no query sees.
+    (Other exact zeros of the reference, such as dQ of a row that sees a
+    single key, are zero only up to rounding on the GPU.)"""
+    Nq, Nk = got[0].shape[2], got[1].shape[2]
+    vis = oracle.visible(np.arange(Nq), Nq, Nk, causal, window)
+    structural = {"dq": ~vis.any(axis=1), "dk": ~vis.any(axis=0), "dv": ~vis.any(axis=0)}
+    for name, g, ref in zip(("dq", "dk", "dv"), got, refs):
+        g = g.float().cpu().numpy()
+        assert np.all(np.isfinite(g)), f"{label}: non-finite {name}"
+        e, idx = max_err(g, ref)
+        bound = max(GRAD_REL_TOL * float(np.abs(ref).max(initial=0.0)), ZERO_REF_FLOOR)
+        assert e <= bound, f"{label}: {name} max err {e:.3e} at {idx} > {bound:.3e}"
+        sel = structural[name]
+        assert np.all(g[:, :, sel] == 0.0), \
+            f"{label}: {name} nonzero on {int(sel.sum())} rows that the mask cuts off"
+
+
+def run_fwd(q, k, v, scale, causal, window):
+    qd, kd, vd = to_dev(q, k, v)
+    o, lse = ea.attn_fwd_masked(qd, kd, vd, scale=scale, causal=causal, window=window)
+    ea.attn_check_status()
+    return o, lse
+
+
+def run_fwd_bwd(q, k, v, do, scale, causal, window):
+    qd, kd, vd, dod = to_dev(q, k, v, do)
+    o, lse = ea.attn_fwd_masked(qd, kd, vd, scale=scale, causal=causal, window=window)
+    dq, dk, dv = ea.attn_bwd_masked(qd, kd, vd, o, lse, dod, scale=scale, causal=causal,
+                                    window=window)
+    ea.attn_check_status()
+    return (o, lse), (dq, dk, dv)
+
+
+# (B, Hq, Hkv, Nq, Nk, d, causal, window)
+FWD_CASES = [
+    # sliding windows at Nq == Nk
+    (1, 2, 2, 300, 300, 128, True, (64, -1)),
+    (1, 2, 2, 300, 300, 128, False, (100, 50)),
+    (1, 2, 2, 300, 300, 64, False, (0, 0)),            # each row sees its own key: O = V
+    (1, 2, 2, 520, 520, 128, False, (255, 255)),
+    (1, 2, 2, 520, 520, 64, False, (-1, 17)),
+    (1, 2, 2, 520, 520, 128, False, (129, -1)),
+    (2, 4, 2, 777, 777, 128, True, (200, 0)),
+    # Nq < Nk (bottom-right: the last query sees every key)
+    (1, 2, 2, 200, 700, 128, True, (-1, -1)),
+    (1, 2, 2, 200, 700, 64, False, (-1, -1)),
+    (1, 2, 1, 200, 700, 128, True, (128, -1)),
+    (1, 4, 4, 1, 1000, 128, True, (-1, -1)),          # one new query over a long prefix
+    (1, 2, 2, 129, 4099, 64, True, (300, -1)),
+    # Nq > Nk: the first Nq - Nk rows see nothing under causal
+    (1, 2, 2, 700, 200, 128, True, (-1, -1)),
+    (1, 2, 2, 700, 200, 64, False, (-1, -1)),
+    (1, 2, 2, 300, 1, 128, True, (-1, -1)),
+    (1, 2, 2, 600, 300, 128, True, (0, 0)),
+    # windows that leave whole tiles without any visible key
+    (1, 2, 2, 300, 1000, 128, True, (50, 0)),
+    (1, 2, 2, 1000, 300, 128, False, (10, 10)),
+    # GQA with windows
+    (2, 8, 2, 384, 640, 128, True, (96, -1)),
+    (1, 6, 3, 257, 257, 64, False, (33, 65)),
+]
+
+
+@pytest.mark.parametrize("case", FWD_CASES,
+                         ids=lambda c: f"B{c[0]}_H{c[1]}_{c[2]}_Nq{c[3]}_Nk{c[4]}_d{c[5]}_c{int(c[6])}_w{c[7][0]}_{c[7][1]}")
+def test_masked_fwd(case):
+    B, Hq, Hkv, Nq, Nk, d, causal, window = case
+    q, k, v = workloads.make_inputs_qk(B, Hq, Hkv, Nq, Nk, d, seed=Nq * 7 + Nk + d,
+                                       with_grad_out=False)
+    scale = d ** -0.5
+    o, lse = run_fwd(q, k, v, scale, causal, window)
+    o_ref, lse_ref = oracle.attention_forward(q, k, v, scale, causal, window=window)
+    assert_masked_fwd_close(o, lse, o_ref, lse_ref, str(case))
+
+
+def test_window_zero_gives_v():
+    """window (0, 0) at Nq == Nk: every row sees exactly its own key, so O = V
+    exactly and lse = scale * q.k."""
+    q, k, v = workloads.make_inputs_qk(1, 2, 2, 300, 300, 128, seed=5, with_grad_out=False)
+    o, _ = run_fwd(q, k, v, 128 ** -0.5, False, (0, 0))
+    assert torch.equal(o.cpu(), v)
+
+
+def test_unmasked_shapes_match_plain_calls_bitwise():
+    """Nq == Nk without a window takes the same kernels as attn_fwd/attn_bwd."""
+    for causal in (False, True):
+        q, k, v, do = workloads.make_inputs_qk(1, 4, 2, 333, 333, 128, seed=11)
+        qd, kd, vd, dod = to_dev(q, k, v, do)
+        o1, l1 = ea.attn_fwd(qd, kd, vd, causal=causal)
+        o2, l2 = ea.attn_fwd_masked(qd, kd, vd, causal=causal, window=(-1, -1))
+        g1 = ea.attn_bwd(qd, kd, vd, o1, l1, dod, causal=causal)
+        g2 = ea.attn_bwd_masked(qd, kd, vd, o2, l2, dod, causal=causal)
+        ea.attn_check_status()
+        assert torch.equal(o1, o2) and torch.equal(l1, l2)
+        for a, b in zip(g1, g2):
+            assert torch.equal(a, b)
+
+
+def test_general_mode_matches_fast_path_on_the_same_mask():
+    """A window wider than the sequence is the unmasked (or causal) problem;
+    it runs the general kernels, whose results must agree with the fast path
+    within rounding (the tile visiting order is the same, so in practice
+    bitwise)."""
+    q, k, v, do = workloads.make_inputs_qk(2, 4, 4, 600, 600, 128, seed=12)
+    qd, kd, vd, dod = to_dev(q, k, v, do)
+    for causal in (False, True):
+        o1, l1 = ea.attn_fwd(qd, kd, vd, causal=causal)
+        o2, l2 = ea.attn_fwd_masked(qd, kd, vd, causal=causal, window=(10_000, 10_000))
+        g1 = ea.attn_bwd(qd, kd, vd, o1, l1, dod, causal=causal)
+        g2 = ea.attn_bwd_masked(qd, kd, vd, o2, l2, dod, causal=causal, window=(10_000, 10_000))
+        ea.attn_check_status()
+        assert (o1.float() - o2.float()).abs().max().item() <= 1e-2
+        assert (l1 - l2).abs().max().item() <= 1e-3
+        for a, b in zip(g1, g2):
+            assert (a.float() - b.float()).abs().max().item() <= 2e-2 * a.float().abs().max().item()
+
+
+BWD_CASES = [
+    (1, 2, 2, 300, 300, 128, True, (64, -1)),
+    (1, 2, 2, 300, 300, 64, False, (40, 70)),
+    (1, 2, 2, 200, 700, 128, True, (-1, -1)),
+    (1, 2, 2, 200, 700, 64, False, (-1, -1)),
+    (1, 2, 2, 700, 200, 128, True, (-1, -1)),          # dQ blocks with no key at all
+    (1, 2, 2, 300, 1000, 128, True, (50, 0)),          # dK/dV tiles no query sees
+    (1, 2, 2, 1000, 300, 64, False, (10, 10)),
+    (2, 8, 2, 384, 640, 128, True, (96, -1)),
+    (1, 4, 1, 1, 777, 128, True, (-1, -1)),
+    (1, 2, 2, 520, 520, 128, False, (0, 0)),
+]
+
+
+@pytest.mark.parametrize("case", BWD_CASES,
+                         ids=lambda c: f"B{c[0]}_H{c[1]}_{c[2]}_Nq{c[3]}_Nk{c[4]}_d{c[5]}_c{int(c[6])}_w{c[7][0]}_{c[7][1]}")
+def test_masked_bwd(case):
+    B, Hq, Hkv, Nq, Nk, d, causal, window = case
+    q, k, v, do = workloads.make_inputs_qk(B, Hq, Hkv, Nq, Nk, d, seed=Nq * 3 + Nk * 5 + d)
+    scale = d ** -0.5
+    (o, lse), got = run_fwd_bwd(q, k, v, do, scale, causal, window)
+    o_ref, lse_ref = oracle.attention_forward(q, k, v, scale, causal, window=window)
+    assert_masked_fwd_close(o, lse, o_ref, lse_ref, str(case))
+    refs = oracle.attention_backward(q, k, v, do, scale, causal, window=window)
+    assert_masked_grads_close(got, refs, str(case), causal, window)
+
+
+def test_masked_bwd_deterministic():
+    q, k, v, do = workloads.make_inputs_qk(1, 4, 2, 500, 900, 128, seed=21)
+    runs = [run_fwd_bwd(q, k, v, do, 128 ** -0.5, True, (200, -1))[1] for _ in range(2)]
+    for a, b in zip(*runs):
+        assert torch.equal(a, b)
+
+
+def test_no_keys():
+    """Nk == 0: O = 0, lse = -inf, dQ = 0 (and no key tensors are read)."""
+    q, k, v, do = workloads.make_inputs_qk(2, 4, 2, 130, 0, 64, seed=3)
+    qd, kd, vd, dod = to_dev(q, k, v, do)
+    o = torch.full_like(qd, 7.0)
+    o, lse = ea.attn_fwd_masked(qd, kd, vd, o=o, causal=True)
+    dq = torch.full_like(qd, 7.0)
+    dq, dk, dv = ea.attn_bwd_masked(qd, kd, vd, o, lse, dod, dq=dq, causal=True)
+    ea.attn_check_status()
+    assert torch.all(o == 0) and torch.all(torch.isneginf(lse)) and torch.all(dq == 0)
+    assert dk.numel() == 0 and dv.numel() == 0
+
+
+def test_no_queries():
+    """Nq == 0 with keys: nothing is written forward; dK = dV = 0 backward."""
+    q, k, v, do = workloads.make_inputs_qk(1, 2, 2, 0, 300, 128, seed=4)
+    qd, kd, vd, dod = to_dev(q, k, v, do)
+    o, lse = ea.attn_fwd_masked(qd, kd, vd)
+    dk = torch.full_like(kd, 3.0)
+    dv = torch.full_like(vd, 3.0)
+    ea.attn_bwd_masked(qd, kd, vd, o, lse, dod, dk=dk, dv=dv)
+    ea.attn_check_status()
+    assert torch.all(dk == 0) and torch.all(dv == 0)
+
+
+def test_large_sliding_window_sampled_rows():
+    """A long sequence with a 1024-key causal window and Nq < Nk (a chunk of
+    new queries over a cached prefix), checked on sampled rows."""
+    B, Hq, Hkv, Nq, Nk, d = 2, 8, 2, 4096, 8192, 128
+    q, k, v = workloads.make_inputs_qk(B, Hq, Hkv, Nq, Nk, d, seed=77, with_grad_out=False)
+    window = (1024, 0)
+    o, lse = run_fwd(q, k, v, d ** -0.5, True, window)
+    o = o.float().cpu().numpy()
+    lse = lse.cpu().numpy()
+    rng = np.random.default_rng(0)
+    rows = np.unique(np.concatenate([[0, 1, 127, 128, 1023, 1024, Nq - 1],
+                                     rng.integers(0, Nq, 40)]))
+    for b, h in ((0, 0), (1, 5), (1, 7)):
+        o_ref, l_ref = oracle.attention_forward_rows(q, k, v, d ** -0.5, True, b, h, rows,
+                                                     window=window)
+        eo, _ = max_err(o[b, h][rows], o_ref)
+        el, _ = max_err(lse[b, h][rows], l_ref)
+        assert eo <= O_TOL and el <= LSE_TOL, (b, h, eo, el)

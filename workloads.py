@@ -95,3 +95,21 @@ def small(name: str, B: int, Hq: int, Hkv: int, N: int, d: int, causal: bool,
           seed: int = 7, q_mult: float = 1.0, backward: bool = True) -> Workload:
     """An edge-case shape for parity tests (ragged N, tiny heads, GQA...)."""
     return Workload(name, B, Hq, Hkv, N, d, causal, q_mult=q_mult, backward=backward, seed=seed)
+
+
+def make_inputs_qk(B: int, Hq: int, Hkv: int, Nq: int, Nk: int, d: int, seed: int,
+                   q_mult: float = 1.0, with_grad_out: bool = True):
+    """(q, k, v[, dO]) with Nq query rows and Nk key rows, CPU bfloat16.
+
+    Same recipe as ``make_inputs``: one generator seeded with ``seed``, draw
+    order Q [B,Hq,Nq,d], K and V [B,Hkv,Nk,d], dO [B,Hq,Nq,d], float32 standard
+    normal rounded once to bfloat16.
+    """
+    g = torch.Generator(device="cpu").manual_seed(seed)
+    q = torch.randn((B, Hq, Nq, d), generator=g, dtype=torch.float32)
+    k = torch.randn((B, Hkv, Nk, d), generator=g, dtype=torch.float32)
+    v = torch.randn((B, Hkv, Nk, d), generator=g, dtype=torch.float32)
+    out = [(q * q_mult).to(torch.bfloat16), k.to(torch.bfloat16), v.to(torch.bfloat16)]
+    if with_grad_out:
+        out.append(torch.randn((B, Hq, Nq, d), generator=g, dtype=torch.float32).to(torch.bfloat16))
+    return tuple(out)
