@@ -380,8 +380,13 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
           float p0 = fast_exp2(x.x);
           float p1 = fast_exp2(x.y);
           if (edge) {
-            if (c < c_lo || c > c_hi) p0 = 0.f;
-            if (c + 1 < c_lo || c + 1 > c_hi) p1 = 0.f;
+            if (MODE == kMaskGeneral) {
+              if (c < c_lo || c > c_hi) p0 = 0.f;
+              if (c + 1 < c_lo || c + 1 > c_hi) p1 = 0.f;
+            } else {                                  // causal diagonal: one-sided
+              if (c < c_lo) p0 = 0.f;
+              if (c + 1 < c_lo) p1 = 0.f;
+            }
           }
           pf[c0 + 2 * e] = p0;
           pf[c0 + 2 * e + 1] = p1;
@@ -670,8 +675,13 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
           float p0 = fast_exp2(x.x);
           float p1 = fast_exp2(x.y);
           if (edge) {
-            if (c < c_lo || c > c_hi) p0 = 0.f;
-            if (c + 1 < c_lo || c + 1 > c_hi) p1 = 0.f;
+            if (MODE == kMaskGeneral) {
+              if (c < c_lo || c > c_hi) p0 = 0.f;
+              if (c + 1 < c_lo || c + 1 > c_hi) p1 = 0.f;
+            } else {                                  // k_lo = 0: one-sided
+              if (c > c_hi) p0 = 0.f;
+              if (c + 1 > c_hi) p1 = 0.f;
+            }
           }
           pf[c0 + 2 * e] = p0;
           pf[c0 + 2 * e + 1] = p1;

@@ -332,12 +332,22 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
       if (edge) {
         const int c_lo = k_lo - kb, c_hi = k_hi - kb;     // keep columns [c_lo, c_hi]
         const uint32_t ninf = f2u(-INFINITY);
+        if (MODE == kMaskGeneral) {
 #pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          if (e < c_lo || e > c_hi) r0[e] = ninf;
-          if (32 + e < c_lo || 32 + e > c_hi) r1[e] = ninf;
-          if (64 + e < c_lo || 64 + e > c_hi) r2[e] = ninf;
-          if (96 + e < c_lo || 96 + e > c_hi) r3[e] = ninf;
+          for (int e = 0; e < 32; ++e) {
+            if (e < c_lo || e > c_hi) r0[e] = ninf;
+            if (32 + e < c_lo || 32 + e > c_hi) r1[e] = ninf;
+            if (64 + e < c_lo || 64 + e > c_hi) r2[e] = ninf;
+            if (96 + e < c_lo || 96 + e > c_hi) r3[e] = ninf;
+          }
+        } else {                                          // k_lo = 0: one-sided
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            if (e > c_hi) r0[e] = ninf;
+            if (32 + e > c_hi) r1[e] = ninf;
+            if (64 + e > c_hi) r2[e] = ninf;
+            if (96 + e > c_hi) r3[e] = ninf;
+          }
         }
       }
       float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
