@@ -21,6 +21,18 @@ written out directly and slowly so it can be checked by eye:
   alignment: ``window = (left, right)`` keeps key ``j`` for query ``i`` iff
   ``i + off - left <= j <= i + off + right`` with ``off = Nk - Nq``. A negative
   side means unbounded. Causal is the case ``right = 0``.
+  Release 2.6 there adds softcapping "as used in Gemma-2 and Grok" without a
+  formula. Read plainly (the form those models use): with ``softcap = c > 0``
+  each scaled logit ``z = scale * q . k`` becomes ``c * tanh(z / c)`` before
+  masking and the softmax; ``c = 0`` turns it off. lse is then the
+  logsumexp of the capped logits.
+* Release 2.0 there renames the unpadded functions to "varlen". Read plainly:
+  a batch of sequences of different lengths is packed token by token with no
+  padding, Q as ``[total_q, Hq, d]`` and K/V as ``[total_k, Hkv, d]``, and
+  ``cu_seqlens_q/k`` (length B+1, starting at 0) give each sequence's first
+  row. Sequence b attends only within itself, with its own ``Nq_b`` and
+  ``Nk_b`` (bottom-right causal alignment and window per sequence). lse is
+  ``[Hq, total_q]``.
 * tokenwerk.de "FlashAttention", section "Was FlashAttention veraendert", and
   unite.ai "Was ist FlashAttention?", the worked example: the method is exact,
   not an approximation. So the oracle is the definition itself. S and P are
@@ -39,7 +51,8 @@ Readings where the pages are silent (each is listed in the design notes):
   gradient of the definition. ``dV = P^T dO``, ``dP = dO V^T`` and
   ``dS = P * (dP - rowsum(P * dP))``. Then ``dQ = scale * dS K`` and
   ``dK = scale * dS^T Q``. Under GQA, dK and dV of a KV head are summed over
-  the query heads that read it.
+  the query heads that read it. With softcapping the chain rule adds the
+  factor ``d(c tanh(z/c))/dz = 1 - tanh(z/c)^2`` to dS.
 
 Inputs may be torch tensors (any dtype, e.g. bfloat16) or numpy arrays. They
 are upcast to float64 once, so the oracle sees the same rounded values the
@@ -110,15 +123,23 @@ def visible(rows, n_q_total: int, n_k: int, causal: bool, window=(-1, -1)) -> np
     return keep
 
 
+def capped(z: np.ndarray, softcap: float) -> np.ndarray:
+    """Softcapping of scaled logits: c * tanh(z / c) for c > 0, identity for c = 0."""
+    if softcap < 0:
+        raise ValueError("softcap must be >= 0")
+    return softcap * np.tanh(z / softcap) if softcap > 0 else z
+
+
 def scores(q: np.ndarray, k: np.ndarray, scale: float, causal: bool,
-           row_offset: int = 0, n_q_total: int | None = None, window=(-1, -1)) -> np.ndarray:
-    """S = (Q K^T) * scale, with masked entries set to -inf.
+           row_offset: int = 0, n_q_total: int | None = None, window=(-1, -1),
+           softcap: float = 0.0) -> np.ndarray:
+    """S = (Q K^T) * scale (softcapped when softcap > 0), masked entries -inf.
 
     ``q`` holds query rows ``row_offset .. row_offset + len(q)`` of a sequence
     of ``n_q_total`` queries (default: just these rows). That is how the
     row-chunked and row-sampled callers keep the causal/window mask right.
     """
-    s = (q @ k.T) * scale
+    s = capped((q @ k.T) * scale, softcap)
     if causal or window[0] >= 0 or window[1] >= 0:
         n_q_total = q.shape[0] if n_q_total is None else n_q_total
         rows = np.arange(row_offset, row_offset + q.shape[0])
@@ -141,14 +162,15 @@ def softmax_rows(s: np.ndarray):
 
 
 def attention_head(q, k, v, scale: float, causal: bool, row_chunk: int = ROW_CHUNK,
-                   window=(-1, -1)):
+                   window=(-1, -1), softcap: float = 0.0):
     """O and lse for one (query head, KV head) pair; q [Nq,d], k/v [Nk,d] float64."""
     n_q = q.shape[0]
     o = np.empty((n_q, v.shape[1]), dtype=np.float64)
     lse = np.empty(n_q, dtype=np.float64)
     for r0 in range(0, n_q, row_chunk):
         r1 = min(n_q, r0 + row_chunk)
-        s = scores(q[r0:r1], k, scale, causal, row_offset=r0, n_q_total=n_q, window=window)
+        s = scores(q[r0:r1], k, scale, causal, row_offset=r0, n_q_total=n_q, window=window,
+                   softcap=softcap)
         p, m, l = softmax_rows(s)
         o[r0:r1] = p @ v
         with np.errstate(divide="ignore"):
@@ -157,10 +179,10 @@ def attention_head(q, k, v, scale: float, causal: bool, row_chunk: int = ROW_CHU
 
 
 def attention_head_rows(q_rows, k, v, scale: float, causal: bool, rows, n_q_total: int,
-                        window=(-1, -1)):
+                        window=(-1, -1), softcap: float = 0.0):
     """O and lse for selected query rows (indices ``rows`` of ``n_q_total``)."""
     rows = np.asarray(rows)
-    s = (q_rows @ k.T) * scale
+    s = capped((q_rows @ k.T) * scale, softcap)
     if causal or window[0] >= 0 or window[1] >= 0:
         s = np.where(visible(rows, n_q_total, k.shape[0], causal, window), s, -np.inf)
     p, m, l = softmax_rows(s)
@@ -169,14 +191,18 @@ def attention_head_rows(q_rows, k, v, scale: float, causal: bool, rows, n_q_tota
     return p @ v, lse
 
 
-def attention_head_bwd(q, k, v, do, scale: float, causal: bool, window=(-1, -1)):
+def attention_head_bwd(q, k, v, do, scale: float, causal: bool, window=(-1, -1),
+                       softcap: float = 0.0):
     """dQ, dK, dV for one head pair, from explicit S and P (no recompute trick)."""
-    s = scores(q, k, scale, causal, window=window)
+    s = scores(q, k, scale, causal, window=window, softcap=softcap)
     p, _, _ = softmax_rows(s)
     dv = p.T @ do
     dp = do @ v.T
     row_dot = np.sum(p * dp, axis=1, keepdims=True)
-    ds = p * (dp - row_dot)
+    ds = p * (dp - row_dot)                      # gradient with respect to the (capped) logits
+    if softcap > 0:
+        t = np.tanh((q @ k.T) * scale / softcap)
+        ds = ds * (1.0 - t * t)                  # chain rule through c * tanh(z / c)
     dq = scale * (ds @ k)
     dk = scale * (ds.T @ q)
     return dq, dk, dv
@@ -192,7 +218,8 @@ def _kv_head(hq: int, n_q_heads: int, n_kv_heads: int) -> int:
     return hq // (n_q_heads // n_kv_heads)
 
 
-def attention_forward(q, k, v, scale: float, causal: bool, window=(-1, -1)):
+def attention_forward(q, k, v, scale: float, causal: bool, window=(-1, -1),
+                      softcap: float = 0.0):
     """O [B,Hq,Nq,d] and lse [B,Hq,Nq] in float64 (K/V may have Nk != Nq rows)."""
     q, k, v = to_f64(q), to_f64(k), to_f64(v)
     B, Hq, Nq, _ = q.shape
@@ -203,22 +230,23 @@ def attention_forward(q, k, v, scale: float, causal: bool, window=(-1, -1)):
         for h in range(Hq):
             hk = _kv_head(h, Hq, Hkv)
             o[b, h], lse[b, h] = attention_head(q[b, h], k[b, hk], v[b, hk], scale, causal,
-                                                window=window)
+                                                window=window, softcap=softcap)
     return o, lse
 
 
 def attention_forward_rows(q, k, v, scale: float, causal: bool, b: int, hq: int, rows,
-                           window=(-1, -1)):
+                           window=(-1, -1), softcap: float = 0.0):
     """O and lse of the listed query rows of head (b, hq), for full-size spot checks."""
     Hq, Nq = q.shape[1], q.shape[2]
     hk = _kv_head(hq, Hq, k.shape[1])
     rows = np.asarray(rows)
     q_rows = to_f64(q[b, hq][rows])
     return attention_head_rows(q_rows, to_f64(k[b, hk]), to_f64(v[b, hk]), scale, causal,
-                               rows, Nq, window=window)
+                               rows, Nq, window=window, softcap=softcap)
 
 
-def attention_backward(q, k, v, do, scale: float, causal: bool, heads=None, window=(-1, -1)):
+def attention_backward(q, k, v, do, scale: float, causal: bool, heads=None, window=(-1, -1),
+                       softcap: float = 0.0):
     """dQ [B,Hq,N,d], dK and dV [B,Hkv,N,d] in float64.
 
     ``heads``: optional list of (b, hkv) KV heads to compute (the others are
@@ -240,7 +268,7 @@ def attention_backward(q, k, v, do, scale: float, causal: bool, heads=None, wind
         dv[b, hk] = 0.0
         for h in range(hk * G, (hk + 1) * G):
             gq, gk, gv = attention_head_bwd(q[b, h], k[b, hk], v[b, hk], do[b, h], scale, causal,
-                                            window=window)
+                                            window=window, softcap=softcap)
             dq[b, h] = gq
             dk[b, hk] += gk
             dv[b, hk] += gv
@@ -299,7 +327,8 @@ def online_softmax_attention_head(q, k, v, scale: float, causal: bool, block: in
 # Brute force for tiny inputs: scalar loops and math.exp, nothing vectorised.
 # --------------------------------------------------------------------------
 
-def attention_bruteforce(q, k, v, scale: float, causal: bool, window=(-1, -1)):
+def attention_bruteforce(q, k, v, scale: float, causal: bool, window=(-1, -1),
+                         softcap: float = 0.0):
     """Pure-Python O and lse for one head; q [Nq][d], k/v [Nk][d] nested lists."""
     n_q, n_k, d_v = len(q), len(k), len(v[0])
     out, lses = [], []
@@ -315,7 +344,10 @@ def attention_bruteforce(q, k, v, scale: float, causal: bool, window=(-1, -1)):
             dot = 0.0
             for c in range(len(q[i])):
                 dot += q[i][c] * k[j][c]
-            logits.append((j, dot * scale))
+            z = dot * scale
+            if softcap > 0:
+                z = softcap * math.tanh(z / softcap)
+            logits.append((j, z))
         if not logits:
             out.append([0.0] * d_v)
             lses.append(-math.inf)
@@ -330,3 +362,68 @@ def attention_bruteforce(q, k, v, scale: float, causal: bool, window=(-1, -1)):
         out.append(row)
         lses.append(big + math.log(total))
     return out, lses
+
+
+# --------------------------------------------------------------------------
+# Varlen (unpadded) batches: sequences packed token by token.
+# --------------------------------------------------------------------------
+
+def _check_cu(cu, total: int, name: str):
+    cu = [int(x) for x in np.asarray(cu).tolist()]
+    if not cu or cu[0] != 0 or cu[-1] != total or any(b < a for a, b in zip(cu, cu[1:])):
+        raise ValueError(f"{name} must start at 0, be non-decreasing and end at {total}")
+    return cu
+
+
+def attention_forward_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, scale: float, causal: bool,
+                             window=(-1, -1), softcap: float = 0.0):
+    """Packed batch: q [total_q, Hq, d], k/v [total_k, Hkv, d] -> O [total_q, Hq, d] and
+    lse [Hq, total_q], float64. Sequence b is rows cu_q[b]:cu_q[b+1] of q and
+    cu_k[b]:cu_k[b+1] of k/v, and attends only within itself."""
+    q, k, v = to_f64(q), to_f64(k), to_f64(v)
+    total_q, Hq, _ = q.shape
+    total_k, Hkv, _ = k.shape
+    cq = _check_cu(cu_seqlens_q, total_q, "cu_seqlens_q")
+    ck = _check_cu(cu_seqlens_k, total_k, "cu_seqlens_k")
+    if len(cq) != len(ck):
+        raise ValueError("cu_seqlens_q and cu_seqlens_k describe different batch sizes")
+    o = np.zeros((total_q, Hq, v.shape[2]))
+    lse = np.full((Hq, total_q), -np.inf)
+    for b in range(len(cq) - 1):
+        q0, q1, k0, k1 = cq[b], cq[b + 1], ck[b], ck[b + 1]
+        if q1 == q0:
+            continue
+        for h in range(Hq):
+            hk = _kv_head(h, Hq, Hkv)
+            if k1 == k0:                      # no keys: O = 0, lse = -inf (already set)
+                continue
+            o[q0:q1, h], lse[h, q0:q1] = attention_head(q[q0:q1, h], k[k0:k1, hk], v[k0:k1, hk],
+                                                        scale, causal, window=window,
+                                                        softcap=softcap)
+    return o, lse
+
+
+def attention_backward_varlen(q, k, v, do, cu_seqlens_q, cu_seqlens_k, scale: float,
+                              causal: bool, window=(-1, -1), softcap: float = 0.0):
+    """dQ [total_q, Hq, d], dK and dV [total_k, Hkv, d] of the packed batch, float64."""
+    q, k, v, do = to_f64(q), to_f64(k), to_f64(v), to_f64(do)
+    total_q, Hq, _ = q.shape
+    total_k, Hkv, _ = k.shape
+    cq = _check_cu(cu_seqlens_q, total_q, "cu_seqlens_q")
+    ck = _check_cu(cu_seqlens_k, total_k, "cu_seqlens_k")
+    dq = np.zeros(q.shape)
+    dk = np.zeros(k.shape)
+    dv = np.zeros(v.shape)
+    for b in range(len(cq) - 1):
+        q0, q1, k0, k1 = cq[b], cq[b + 1], ck[b], ck[b + 1]
+        if q1 == q0 or k1 == k0:
+            continue
+        for h in range(Hq):
+            hk = _kv_head(h, Hq, Hkv)
+            gq, gk, gv = attention_head_bwd(q[q0:q1, h], k[k0:k1, hk], v[k0:k1, hk],
+                                            do[q0:q1, h], scale, causal, window=window,
+                                            softcap=softcap)
+            dq[q0:q1, h] = gq
+            dk[k0:k1, hk] += gk
+            dv[k0:k1, hk] += gv
+    return dq, dk, dv
