@@ -9,7 +9,9 @@ sm_100 part, every call raises.
 Layout: q, o, dO, dq are [B, Hq, Nq, d]. k, v, dk, dv are [B, Hkv, Nk, d].
 All are contiguous bfloat16 CUDA tensors. lse is [B, Hq, Nq] float32.
 ``attn_fwd``/``attn_bwd`` need Nq == Nk; the ``*_masked`` calls take
-Nq != Nk (bottom-right causal alignment) and a sliding window.
+Nq != Nk (bottom-right causal alignment), a sliding window and softcapping.
+The ``*_varlen`` calls take a packed batch: q/o/dO/dq [total_q, Hq, d],
+k/v/dk/dv [total_k, Hkv, d], lse [Hq, total_q], with int32 cu_seqlens.
 """
 from __future__ import annotations
 
@@ -33,9 +35,14 @@ SIGNATURES = {
     "attn_bwd_workspace_size": (_SZ, [_I, _I, _I, _I]),
     "attn_bwd_noalloc": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P,
                               _I, _I, _I, _I, _I, _F, _I, _P]),
-    "attn_fwd_masked": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _I, _I, _I, _P]),
+    "attn_fwd_masked": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _I, _I, _I, _F,
+                             _P]),
     "attn_bwd_masked": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _SZ,
-                             _I, _I, _I, _I, _I, _I, _F, _I, _I, _I, _P]),
+                             _I, _I, _I, _I, _I, _I, _F, _I, _I, _I, _F, _P]),
+    "attn_fwd_varlen": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _F,
+                             _I, _I, _I, _F, _P]),
+    "attn_bwd_varlen": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _SZ,
+                             _I, _I, _I, _I, _I, _I, _I, _I, _F, _I, _I, _I, _F, _P]),
     "attn_check_status": (_I, [_P]),
     "attn_selftest_wait_timeout": (_I, [_P]),
     "attn_get_last_error": (ctypes.c_char_p, []),
@@ -191,12 +198,20 @@ def _window(window):
     return max(left, -1), max(right, -1)
 
 
+def _softcap(softcap):
+    c = 0.0 if softcap is None else float(softcap)
+    if not math.isfinite(c) or c < 0:
+        raise ValueError(f"softcap must be finite and >= 0, got {softcap}")
+    return c
+
+
 def attn_fwd_masked(q, k, v, o=None, lse=None, scale=None, causal=False, window=(-1, -1),
-                    stream=None):
+                    softcap=0.0, stream=None):
     """Forward with Nq = q.shape[2] queries, Nk = k.shape[2] keys and a sliding
     window (left, right); a negative side is unbounded. Query i sees key j iff
     i + Nk - Nq - left <= j <= i + Nk - Nq + right (and j <= i + Nk - Nq when
-    causal). Rows that see no key get o = 0, lse = -inf. Returns (o, lse)."""
+    causal). softcap = c > 0 caps each scaled logit z to c * tanh(z / c).
+    Rows that see no key get o = 0, lse = -inf. Returns (o, lse)."""
     import torch
     B, Hq, Nq, d = q.shape
     Hkv, Nk = k.shape[1], k.shape[2]
@@ -215,13 +230,14 @@ def attn_fwd_masked(q, k, v, o=None, lse=None, scale=None, causal=False, window=
     lib = load_library()
     _check(lib.attn_fwd_masked(_dev_ptr(q, "q"), _dev_ptr(k, "k"), _dev_ptr(v, "v"),
                                _dev_ptr(o, "o"), _dev_ptr(lse, "lse"), B, Hq, Hkv, Nq, Nk, d,
-                               scale, int(bool(causal)), wl, wr, _stream_handle(stream)))
+                               scale, int(bool(causal)), wl, wr, _softcap(softcap),
+                               _stream_handle(stream)))
     return o, lse
 
 
 def attn_bwd_masked(q, k, v, o, lse, dO, dq=None, dk=None, dv=None, workspace=None, scale=None,
-                    causal=False, window=(-1, -1), stream=None):
-    """Backward of attn_fwd_masked with the same causal/window; returns (dq, dk, dv)."""
+                    causal=False, window=(-1, -1), softcap=0.0, stream=None):
+    """Backward of attn_fwd_masked with the same causal/window/softcap; returns (dq, dk, dv)."""
     import torch
     B, Hq, Nq, d = q.shape
     Hkv, Nk = k.shape[1], k.shape[2]
@@ -250,6 +266,92 @@ def attn_bwd_masked(q, k, v, o, lse, dO, dq=None, dk=None, dv=None, workspace=No
                                _dev_ptr(workspace, "workspace"),
                                workspace.numel() * workspace.element_size(),
                                B, Hq, Hkv, Nq, Nk, d, scale, int(bool(causal)), wl, wr,
+                               _softcap(softcap), _stream_handle(stream)))
+    return dq, dk, dv
+
+
+def _check_cu(cu, name, device):
+    import torch
+    if not isinstance(cu, torch.Tensor) or cu.dtype != torch.int32 or cu.dim() != 1:
+        raise TypeError(f"{name} must be a 1-D int32 tensor")
+    if not cu.is_cuda or cu.device != device or not cu.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous CUDA tensor on {device}")
+    return ctypes.c_void_p(cu.data_ptr())
+
+
+def attn_fwd_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, max_seqlen_k, o=None,
+                    lse=None, scale=None, causal=False, window=(-1, -1), softcap=0.0, stream=None):
+    """Packed batch forward: q [total_q, Hq, d], k/v [total_k, Hkv, d], int32
+    cu_seqlens of length B + 1 on the device. Returns (o [total_q, Hq, d],
+    lse [Hq, total_q]). Offsets are checked on the GPU: invalid ones make the
+    next attn_check_status() raise."""
+    import torch
+    total_q, Hq, d = q.shape
+    total_k, Hkv = k.shape[0], k.shape[1]
+    if k.shape != (total_k, Hkv, d) or v.shape != k.shape:
+        raise ValueError("k/v must be [total_k, Hkv, d] with q's d")
+    if cu_seqlens_q.shape != cu_seqlens_k.shape:
+        raise ValueError("cu_seqlens_q and cu_seqlens_k must have the same length (B + 1)")
+    B = cu_seqlens_q.shape[0] - 1
+    cq = _check_cu(cu_seqlens_q, "cu_seqlens_q", q.device)
+    ck = _check_cu(cu_seqlens_k, "cu_seqlens_k", q.device)
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _check_dtype(t, torch.bfloat16, n)
+    o = torch.empty_like(q) if o is None else o
+    lse = torch.empty((Hq, total_q), dtype=torch.float32, device=q.device) if lse is None else lse
+    _check_dtype(o, torch.bfloat16, "o")
+    _check_dtype(lse, torch.float32, "lse")
+    if o.shape != q.shape or lse.shape != (Hq, total_q):
+        raise ValueError("o/lse shape mismatch")
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    wl, wr = _window(window)
+    lib = load_library()
+    _check(lib.attn_fwd_varlen(_dev_ptr(q, "q"), _dev_ptr(k, "k"), _dev_ptr(v, "v"),
+                               _dev_ptr(o, "o"), _dev_ptr(lse, "lse"), cq, ck, B, Hq, Hkv,
+                               total_q, total_k, int(max_seqlen_q), int(max_seqlen_k), d, scale,
+                               int(bool(causal)), wl, wr, _softcap(softcap),
+                               _stream_handle(stream)))
+    return o, lse
+
+
+def attn_bwd_varlen(q, k, v, o, lse, dO, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, max_seqlen_k,
+                    dq=None, dk=None, dv=None, workspace=None, scale=None, causal=False,
+                    window=(-1, -1), softcap=0.0, stream=None):
+    """Backward of attn_fwd_varlen with the same arguments; returns (dq, dk, dv)."""
+    import torch
+    total_q, Hq, d = q.shape
+    total_k, Hkv = k.shape[0], k.shape[1]
+    if k.shape != (total_k, Hkv, d) or v.shape != k.shape or o.shape != q.shape \
+            or dO.shape != q.shape or lse.shape != (Hq, total_q):
+        raise ValueError("shape mismatch among q, k, v, o, lse, dO")
+    if cu_seqlens_q.shape != cu_seqlens_k.shape:
+        raise ValueError("cu_seqlens_q and cu_seqlens_k must have the same length (B + 1)")
+    B = cu_seqlens_q.shape[0] - 1
+    cq = _check_cu(cu_seqlens_q, "cu_seqlens_q", q.device)
+    ck = _check_cu(cu_seqlens_k, "cu_seqlens_k", q.device)
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (o, "o"), (dO, "dO")):
+        _check_dtype(t, torch.bfloat16, n)
+    _check_dtype(lse, torch.float32, "lse")
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    for t, n, ref in ((dq, "dq", q), (dk, "dk", k), (dv, "dv", v)):
+        _check_dtype(t, torch.bfloat16, n)
+        if t.shape != ref.shape:
+            raise ValueError(f"{n} shape mismatch")
+    need = attn_bwd_workspace_size(B, Hq, int(max_seqlen_q), d)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    wl, wr = _window(window)
+    lib = load_library()
+    _check(lib.attn_bwd_varlen(_dev_ptr(q, "q"), _dev_ptr(k, "k"), _dev_ptr(v, "v"),
+                               _dev_ptr(o, "o"), _dev_ptr(lse, "lse"), _dev_ptr(dO, "dO"),
+                               _dev_ptr(dq, "dq"), _dev_ptr(dk, "dk"), _dev_ptr(dv, "dv"), cq, ck,
+                               _dev_ptr(workspace, "workspace"),
+                               workspace.numel() * workspace.element_size(), B, Hq, Hkv, total_q,
+                               total_k, int(max_seqlen_q), int(max_seqlen_k), d, scale,
+                               int(bool(causal)), wl, wr, _softcap(softcap),
                                _stream_handle(stream)))
     return dq, dk, dv
 

@@ -136,15 +136,17 @@ attn_status ensure_init() {
   if (g_init_status != ATTN_OK) return fail(g_init_status, "%s", g_init_msg);
   return ATTN_OK;
 }
-
-// 3-D tensor map over a contiguous [BH, N, d] bf16 tensor with a box of
-// 64 x 128 x 1 (one 128-row, 128-byte-wide column block) and 128-byte
-// swizzle. Rows past N of a head read as zeros, never as the next head.
-attn_status make_map(CUtensorMap* map, const void* base, int d, int N, int BH) {
-  cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N),
-                        static_cast<cuuint64_t>(BH)};
-  cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2,
-                           static_cast<cuuint64_t>(d) * 2 * static_cast<cuuint64_t>(N)};
+// 3-D tensor map (d, rows, z) over a bf16 tensor, with a box of 64 x 128 x 1
+// (one 128-row, 128-byte-wide column block) and 128-byte swizzle. Row and z
+// strides are in elements. Fixed-length [B*H, N, d]: rows = N, z = B*H,
+// row stride d, z stride N*d. Packed [total, H, d]: rows = total, z = H, row
+// stride H*d, z stride d. Rows past `rows` read as zeros.
+attn_status make_map(CUtensorMap* map, const void* base, int d, long long rows, long long zdim,
+                     long long row_stride, long long z_stride) {
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(rows),
+                        static_cast<cuuint64_t>(zdim)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(row_stride) * 2,
+                           static_cast<cuuint64_t>(z_stride) * 2};
   cuuint32_t box[3] = {64, 128, 1};
   cuuint32_t estr[3] = {1, 1, 1};
   CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims,
@@ -199,28 +201,41 @@ attn_status check_shape(int B, int Hq, int Hkv, int N, int d, float scale, bool*
 // Which keys each query row sees: the three kernel mask modes and the window
 // bounds they use. window_left/right < 0 is unbounded; causal caps the right
 // side at 0. Same-length problems without a left window keep the unmasked
-// and causal fast paths.
+// and causal fast paths. Packed batches and softcapping always run the
+// general mode (its bounds are per sequence; the softcap variant exists only
+// there). The kernels set the offset Nk - Nq per sequence.
 struct MaskSpec {
   int mode;
+  bool softcap;
   attn::KeyWindow win;
 };
 
-MaskSpec mask_spec(int Nq, int Nk, int causal, int window_left, int window_right) {
+MaskSpec mask_spec(int Nq, int Nk, int causal, int window_left, int window_right, bool packed,
+                   float softcap) {
   using namespace attn;
   const int wl = window_left < 0 ? kUnbounded : std::min(window_left, kUnbounded);
   int wr = window_right < 0 ? kUnbounded : std::min(window_right, kUnbounded);
   if (causal) wr = 0;
-  const bool plain = Nq == Nk && wl == kUnbounded && (causal || wr == kUnbounded);
+  const bool plain = !packed && softcap == 0.f && Nq == Nk && wl == kUnbounded &&
+                     (causal || wr == kUnbounded);
   const int mode = plain ? (causal ? kMaskCausal : kMaskNone) : kMaskGeneral;
-  return MaskSpec{mode, KeyWindow{Nk - Nq, wl, wr}};
+  return MaskSpec{mode, softcap > 0.f, KeyWindow{Nk - Nq, wl, wr}};
 }
 
-template <int D, int MODE>
+// Everything a launch needs besides the tensor maps.
+struct Problem {
+  int B, Hq, Hkv, d;
+  attn::SeqGeom geom;
+  float scale;
+  MaskSpec mask;
+  attn::Softcap cap;
+};
+
+template <int D, int MODE, int FEAT>
 attn_status launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
-                       void* o, float* lse, int B, int Hq, int Hkv, int Nq, int Nk, float scale,
-                       attn::KeyWindow win, cudaStream_t stream) {
+                       void* o, float* lse, const Problem& p, cudaStream_t stream) {
   using Cfg = attn::FwdCfg<D>;
-  auto kern = attn::fwd_kernel<D, MODE>;
+  auto kern = attn::fwd_kernel<D, MODE, FEAT>;
   static std::once_flag attr_once;
   static cudaError_t attr_err = cudaSuccess;
   static int launch_regs = 0;
@@ -237,13 +252,14 @@ attn_status launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUten
   if (launch_regs != attn::kFwdRegsLaunch)
     return fail(ATTN_ERR_CUDA, "fwd kernel built with %d registers/thread, expected %d",
                 launch_regs, attn::kFwdRegsLaunch);
-  const long long blocks = static_cast<long long>(B) * Hq * ((Nq + 255) / 256);
+  const long long blocks = static_cast<long long>(p.B) * p.Hq * ((p.geom.Nq + 255) / 256);
   if (blocks > 0x7FFFFFFFLL) return fail(ATTN_ERR_ARG, "problem too large for one launch");
   dim3 grid(static_cast<unsigned>(blocks));
-  const float scale_log2 = scale * 1.4426950408889634f;
+  const float scale_log2 = p.scale * 1.4426950408889634f;
   ProfScope ps(kProfFwd, stream);
   kern<<<grid, Cfg::kThreads, Cfg::kSmemAlloc, stream>>>(
-      mq, mk, mv, static_cast<__nv_bfloat16*>(o), lse, Hq, Hq / Hkv, Nq, Nk, scale_log2, win);
+      mq, mk, mv, static_cast<__nv_bfloat16*>(o), lse, p.Hq, p.Hq / p.Hkv, p.geom, scale_log2,
+      p.mask.win, p.cap);
   ps.end();
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "fwd kernel launch");
@@ -266,34 +282,32 @@ struct BwdArgs {
   const void* dO;
   void *dq, *dk, *dv;
   float *L, *Dv;
-  int B, Hq, Hkv, Nq, Nk;
-  float scale;
-  attn::KeyWindow win;
 };
 
-template <int D, int MODE>
-attn_status launch_bwd(const BwdArgs& a, cudaStream_t stream) {
+template <int D, int MODE, int FEAT>
+attn_status launch_bwd(const BwdArgs& a, const Problem& p, cudaStream_t stream) {
   using namespace attn;
-  const int Npad = pad128(a.Nq);
-  const int group = a.Hq / a.Hkv;
-  const float scale_log2 = a.scale * kLog2e;
+  const int Npad = pad128(p.geom.Nq);
+  const int group = p.Hq / p.Hkv;
+  const float scale_log2 = p.scale * kLog2e;
 
-  const long long rows = static_cast<long long>(a.B) * a.Hq * Npad;
-  const long long g1 = static_cast<long long>(pad128(a.Nk) / 128) * a.B * a.Hkv;
-  const long long g2 = static_cast<long long>(Npad / 128) * a.B * a.Hq;
-  if (rows / 32 > 0x7FFFFFFFLL) return fail(ATTN_ERR_ARG, "problem too large for one launch");
+  const long long rows = static_cast<long long>(p.B) * p.Hq * Npad;
+  const long long g1 = static_cast<long long>(pad128(p.geom.Nk) / 128) * p.B * p.Hkv;
+  const long long g2 = static_cast<long long>(Npad / 128) * p.B * p.Hq;
+  if (rows / 32 > 0x7FFFFFFFLL || g1 > 0x7FFFFFFFLL || g2 > 0x7FFFFFFFLL)
+    return fail(ATTN_ERR_ARG, "problem too large for one launch");
   ProfScope p0(kProfBwdPre, stream);
   bwd_pre_kernel<D><<<static_cast<unsigned>(rows / 32), 256, 0, stream>>>(
       static_cast<const __nv_bfloat16*>(a.o), static_cast<const __nv_bfloat16*>(a.dO), a.lse,
-      a.L, a.Dv, a.Nq, Npad);
+      a.L, a.Dv, p.Hq, p.geom, Npad);
   p0.end();
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "bwd preprocess launch");
 
   static std::once_flag o1, o2;
   static cudaError_t e1 = cudaSuccess, e2 = cudaSuccess;
-  auto k1 = bwd_dkdv_kernel<D, MODE>;
-  auto k2 = bwd_dq_kernel<D, MODE>;
+  auto k1 = bwd_dkdv_kernel<D, MODE, FEAT>;
+  auto k2 = bwd_dq_kernel<D, MODE, FEAT>;
   if ((e = set_smem_once(k1, DkdvCfg<D>::kSmemAlloc, o1, e1)) != cudaSuccess)
     return cuda_fail(e, "cudaFuncSetAttribute(dkdv)");
   if ((e = set_smem_once(k2, DqCfg<D>::kSmemAlloc, o2, e2)) != cudaSuccess)
@@ -302,14 +316,14 @@ attn_status launch_bwd(const BwdArgs& a, cudaStream_t stream) {
   ProfScope p1(kProfBwdDkdv, stream);
   k1<<<dim3(static_cast<unsigned>(g1)), DkdvCfg<D>::kThreads, DkdvCfg<D>::kSmemAlloc, stream>>>(
       a.mq, a.mk, a.mv, a.mdo, a.L, a.Dv, static_cast<__nv_bfloat16*>(a.dk),
-      static_cast<__nv_bfloat16*>(a.dv), a.Hq, group, a.Nq, a.Nk, Npad, scale_log2, a.scale,
-      a.win);
+      static_cast<__nv_bfloat16*>(a.dv), p.Hq, group, p.geom, Npad, scale_log2, p.scale,
+      p.mask.win, p.cap);
   p1.end();
   if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "bwd dK/dV launch");
   ProfScope p2(kProfBwdDq, stream);
   k2<<<dim3(static_cast<unsigned>(g2)), DqCfg<D>::kThreads, DqCfg<D>::kSmemAlloc, stream>>>(
-      a.mq, a.mk, a.mv, a.mdo, a.L, a.Dv, static_cast<__nv_bfloat16*>(a.dq), a.Hq, group, a.Nq,
-      a.Nk, Npad, scale_log2, a.scale, a.win);
+      a.mq, a.mk, a.mv, a.mdo, a.L, a.Dv, static_cast<__nv_bfloat16*>(a.dq), p.Hq, group, p.geom,
+      Npad, scale_log2, p.scale, p.mask.win, p.cap);
   p2.end();
   if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "bwd dQ launch");
   return ATTN_OK;
@@ -375,35 +389,31 @@ __global__ void fill_neg_inf_kernel(float* p, long long n) {
 
 template <int D>
 attn_status dispatch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
-                         void* o, float* lse, int B, int Hq, int Hkv, int Nq, int Nk, float scale,
-                         const MaskSpec& m, cudaStream_t stream) {
+                         void* o, float* lse, const Problem& p, cudaStream_t stream) {
   using namespace attn;
-  if (m.mode == kMaskNone)
-    return launch_fwd<D, kMaskNone>(mq, mk, mv, o, lse, B, Hq, Hkv, Nq, Nk, scale, m.win, stream);
-  if (m.mode == kMaskCausal)
-    return launch_fwd<D, kMaskCausal>(mq, mk, mv, o, lse, B, Hq, Hkv, Nq, Nk, scale, m.win,
-                                      stream);
-  return launch_fwd<D, kMaskGeneral>(mq, mk, mv, o, lse, B, Hq, Hkv, Nq, Nk, scale, m.win, stream);
+  if (p.mask.mode == kMaskNone) return launch_fwd<D, kMaskNone, 0>(mq, mk, mv, o, lse, p, stream);
+  if (p.mask.mode == kMaskCausal)
+    return launch_fwd<D, kMaskCausal, 0>(mq, mk, mv, o, lse, p, stream);
+  const bool packed = p.geom.cu_q != nullptr;
+  if (packed && p.mask.softcap)
+    return launch_fwd<D, kMaskGeneral, kFeatPacked | kFeatSoftcap>(mq, mk, mv, o, lse, p, stream);
+  if (packed) return launch_fwd<D, kMaskGeneral, kFeatPacked>(mq, mk, mv, o, lse, p, stream);
+  if (p.mask.softcap)
+    return launch_fwd<D, kMaskGeneral, kFeatSoftcap>(mq, mk, mv, o, lse, p, stream);
+  return launch_fwd<D, kMaskGeneral, 0>(mq, mk, mv, o, lse, p, stream);
 }
 
 template <int D>
-attn_status dispatch_bwd(const BwdArgs& a, int mode, cudaStream_t stream) {
+attn_status dispatch_bwd(const BwdArgs& a, const Problem& p, cudaStream_t stream) {
   using namespace attn;
-  if (mode == kMaskNone) return launch_bwd<D, kMaskNone>(a, stream);
-  if (mode == kMaskCausal) return launch_bwd<D, kMaskCausal>(a, stream);
-  return launch_bwd<D, kMaskGeneral>(a, stream);
-}
-
-attn_status check_common(int B, int Hq, int Hkv, int Nq, int Nk, int d, float scale, int causal,
-                         bool* no_rows, bool* no_keys) {
-  bool eq = false, ek = false;
-  attn_status st = check_shape(B, Hq, Hkv, Nq, d, scale, &eq);
-  if (st != ATTN_OK) return st;
-  if ((st = check_shape(B, Hq, Hkv, Nk, d, scale, &ek)) != ATTN_OK) return st;
-  if (causal != 0 && causal != 1) return fail(ATTN_ERR_ARG, "causal must be 0 or 1");
-  *no_rows = eq;
-  *no_keys = ek;
-  return ATTN_OK;
+  if (p.mask.mode == kMaskNone) return launch_bwd<D, kMaskNone, 0>(a, p, stream);
+  if (p.mask.mode == kMaskCausal) return launch_bwd<D, kMaskCausal, 0>(a, p, stream);
+  const bool packed = p.geom.cu_q != nullptr;
+  if (packed && p.mask.softcap)
+    return launch_bwd<D, kMaskGeneral, kFeatPacked | kFeatSoftcap>(a, p, stream);
+  if (packed) return launch_bwd<D, kMaskGeneral, kFeatPacked>(a, p, stream);
+  if (p.mask.softcap) return launch_bwd<D, kMaskGeneral, kFeatSoftcap>(a, p, stream);
+  return launch_bwd<D, kMaskGeneral, 0>(a, p, stream);
 }
 
 attn_status check_args(const void* const* ptrs, const char* const* names, const bool* used,
@@ -429,58 +439,152 @@ attn_status check_used_ptrs(const void* const* ptrs, const char* const* names, c
   return check_ptrs(p, nm, m);
 }
 
-attn_status fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, int B,
-                     int Hq, int Hkv, int Nq, int Nk, int d, float scale, int causal,
-                     int window_left, int window_right, cudaStream_t stream) {
-  g_last_error[0] = '\0';
-  bool no_rows = false, no_keys = false;
-  attn_status st = check_common(B, Hq, Hkv, Nq, Nk, d, scale, causal, &no_rows, &no_keys);
+attn_status check_mask_args(int causal, float softcap) {
+  if (causal != 0 && causal != 1) return fail(ATTN_ERR_ARG, "causal must be 0 or 1");
+  if (!(softcap >= 0.f) || !std::isfinite(softcap))
+    return fail(ATTN_ERR_ARG, "softcap must be finite and >= 0 (got %g)", (double)softcap);
+  return ATTN_OK;
+}
+
+attn::Softcap softcap_consts(float scale, float softcap) {
+  if (softcap <= 0.f) return attn::Softcap{0.f, 0.f};
+  return attn::Softcap{2.0f * scale * attn::kLog2e / softcap, softcap * attn::kLog2e};
+}
+
+// How Q-side and K-side tensors are laid out: TMA map shapes and sizes.
+struct Layout {
+  long long q_rows, q_z, q_rs, q_zs;   // rows, z extent, row stride, z stride (elements)
+  long long k_rows, k_z, k_rs, k_zs;
+  long long q_elems, k_elems, lse_elems;
+};
+
+// Fixed length: [B, H, N, d], lse [B, Hq, Nq].
+void fixed_problem(int B, int Hq, int Hkv, int Nq, int Nk, int d, float scale, int causal, int wl,
+                   int wr, float softcap, Problem* p, Layout* L) {
+  p->B = B; p->Hq = Hq; p->Hkv = Hkv; p->d = d; p->scale = scale;
+  p->geom = attn::SeqGeom{nullptr, nullptr, Nq, Nk, 0, 0, static_cast<long long>(Nq) * d, d,
+                          static_cast<long long>(Nk) * d, d, Nq};
+  p->mask = mask_spec(Nq, Nk, causal, wl, wr, false, softcap);
+  p->cap = softcap_consts(scale, softcap);
+  *L = Layout{Nq, static_cast<long long>(B) * Hq, d, static_cast<long long>(Nq) * d,
+              Nk, static_cast<long long>(B) * Hkv, d, static_cast<long long>(Nk) * d,
+              static_cast<long long>(B) * Hq * Nq * d, static_cast<long long>(B) * Hkv * Nk * d,
+              static_cast<long long>(B) * Hq * Nq};
+}
+
+// Packed: [total, H, d], lse [Hq, total_q], sequences at cu_q / cu_k.
+void packed_problem(const int* cu_q, const int* cu_k, int B, int Hq, int Hkv, int total_q,
+                    int total_k, int max_q, int max_k, int d, float scale, int causal, int wl,
+                    int wr, float softcap, Problem* p, Layout* L) {
+  p->B = B; p->Hq = Hq; p->Hkv = Hkv; p->d = d; p->scale = scale;
+  p->geom = attn::SeqGeom{cu_q, cu_k, max_q, max_k, total_q, total_k, d,
+                          static_cast<long long>(Hq) * d, d, static_cast<long long>(Hkv) * d,
+                          total_q};
+  p->mask = mask_spec(max_q, max_k, causal, wl, wr, true, softcap);
+  p->cap = softcap_consts(scale, softcap);
+  *L = Layout{total_q, Hq, static_cast<long long>(Hq) * d, d,
+              total_k, Hkv, static_cast<long long>(Hkv) * d, d,
+              static_cast<long long>(total_q) * Hq * d, static_cast<long long>(total_k) * Hkv * d,
+              static_cast<long long>(Hq) * total_q};
+}
+
+// Offsets arrays: null and alignment (host only), then, with a device
+// present, that they are device memory.
+attn_status check_offsets_args(const int* cu_q, const int* cu_k) {
+  const void* ptrs[2] = {cu_q, cu_k};
+  const char* names[2] = {"cu_seqlens_q", "cu_seqlens_k"};
+  for (int i = 0; i < 2; ++i) {
+    if (ptrs[i] == nullptr) return fail(ATTN_ERR_ARG, "%s is null", names[i]);
+    if ((reinterpret_cast<uintptr_t>(ptrs[i]) & 3u) != 0)
+      return fail(ATTN_ERR_ARG, "%s is not 4-byte aligned", names[i]);
+  }
+  return ATTN_OK;
+}
+
+attn_status check_offsets(const int* cu_q, const int* cu_k) {
+  const void* ptrs[2] = {cu_q, cu_k};
+  const char* names[2] = {"cu_seqlens_q", "cu_seqlens_k"};
+  for (int i = 0; i < 2; ++i) {
+    cudaPointerAttributes pa;
+    cudaError_t e = cudaPointerGetAttributes(&pa, ptrs[i]);
+    if (e != cudaSuccess) {
+      cudaGetLastError();
+      return fail(ATTN_ERR_ARG, "%s is not a CUDA pointer (%s)", names[i], cudaGetErrorName(e));
+    }
+    if (pa.type != cudaMemoryTypeDevice && pa.type != cudaMemoryTypeManaged)
+      return fail(ATTN_ERR_ARG, "%s is not device memory", names[i]);
+  }
+  return ATTN_OK;
+}
+
+// Packed-batch argument checks (host side; offsets are checked on the GPU).
+attn_status check_packed(int B, int Hq, int Hkv, int total_q, int total_k, int max_q, int max_k,
+                         int d, float scale, bool* no_rows, bool* no_keys) {
+  bool e1 = false, e2 = false;
+  attn_status st = check_shape(B, Hq, Hkv, max_q, d, scale, &e1);
   if (st != ATTN_OK) return st;
-  if (no_rows) return ATTN_OK;                 // B == 0 or Nq == 0: nothing to write
+  if ((st = check_shape(B, Hq, Hkv, max_k, d, scale, &e2)) != ATTN_OK) return st;
+  if (total_q < 0 || total_k < 0)
+    return fail(ATTN_ERR_ARG, "total_q and total_k must be >= 0 (got %d, %d)", total_q, total_k);
+  if ((total_q > 0 && max_q == 0) || (total_k > 0 && max_k == 0))
+    return fail(ATTN_ERR_ARG, "max_seqlen must be >= 1 when the packed tensor has rows");
+  if (static_cast<long long>(total_q) * Hq > 0x7FFFFFFFLL ||
+      static_cast<long long>(total_k) * Hkv > 0x7FFFFFFFLL)
+    return fail(ATTN_ERR_ARG, "packed tensors too large (total * H must be < 2^31)");
+  *no_rows = B == 0 || total_q == 0;
+  *no_keys = B == 0 || total_k == 0;
+  return ATTN_OK;
+}
+
+attn_status fwd_run(const void* q, const void* k, const void* v, void* o, float* lse,
+                    const int* cu_q, const int* cu_k, const Problem& p, const Layout& L,
+                    bool no_rows, bool no_keys, cudaStream_t stream) {
+  if (no_rows) return ATTN_OK;                 // no query rows: nothing to write
   const void* ptrs[5] = {q, k, v, o, lse};
   const char* names[5] = {"q", "k", "v", "o", "lse"};
   const bool used[5] = {!no_keys, !no_keys, !no_keys, true, true};
-  if ((st = check_args(ptrs, names, used, 5)) != ATTN_OK) return st;
+  const bool packed = p.geom.cu_q != nullptr || cu_q != nullptr || cu_k != nullptr;
+  attn_status st = check_args(ptrs, names, used, 5);
+  if (st != ATTN_OK) return st;
+  if (packed && (st = check_offsets_args(cu_q, cu_k)) != ATTN_OK) return st;
   if ((st = ensure_init()) != ATTN_OK) return st;
   if ((st = check_used_ptrs(ptrs, names, used, 5)) != ATTN_OK) return st;
+  if (packed && (st = check_offsets(cu_q, cu_k)) != ATTN_OK) return st;
   if (no_keys) {
-    // Nk == 0: every row sees no key, so O = 0 and lse = -inf.
-    const long long rows = static_cast<long long>(B) * Hq * Nq;
-    cudaError_t e = cudaMemsetAsync(o, 0, static_cast<size_t>(rows) * d * 2, stream);
+    // No keys at all: every row sees no key, so O = 0 and lse = -inf.
+    cudaError_t e = cudaMemsetAsync(o, 0, static_cast<size_t>(L.q_elems) * 2, stream);
     if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(o)");
-    fill_neg_inf_kernel<<<static_cast<unsigned>(std::min<long long>((rows + 255) / 256, 4096)),
-                          256, 0, stream>>>(lse, rows);
+    fill_neg_inf_kernel<<<static_cast<unsigned>(std::min<long long>((L.lse_elems + 255) / 256, 4096)),
+                          256, 0, stream>>>(lse, L.lse_elems);
     if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "lse fill launch");
     return ATTN_OK;
   }
   CUtensorMap mq, mk, mv;
-  if ((st = make_map(&mq, q, d, Nq, B * Hq)) != ATTN_OK) return st;
-  if ((st = make_map(&mk, k, d, Nk, B * Hkv)) != ATTN_OK) return st;
-  if ((st = make_map(&mv, v, d, Nk, B * Hkv)) != ATTN_OK) return st;
-  const MaskSpec m = mask_spec(Nq, Nk, causal, window_left, window_right);
-  if (d == 64) return dispatch_fwd<64>(mq, mk, mv, o, lse, B, Hq, Hkv, Nq, Nk, scale, m, stream);
-  return dispatch_fwd<128>(mq, mk, mv, o, lse, B, Hq, Hkv, Nq, Nk, scale, m, stream);
+  if ((st = make_map(&mq, q, p.d, L.q_rows, L.q_z, L.q_rs, L.q_zs)) != ATTN_OK) return st;
+  if ((st = make_map(&mk, k, p.d, L.k_rows, L.k_z, L.k_rs, L.k_zs)) != ATTN_OK) return st;
+  if ((st = make_map(&mv, v, p.d, L.k_rows, L.k_z, L.k_rs, L.k_zs)) != ATTN_OK) return st;
+  if (p.d == 64) return dispatch_fwd<64>(mq, mk, mv, o, lse, p, stream);
+  return dispatch_fwd<128>(mq, mk, mv, o, lse, p, stream);
 }
 
-// Backward shared by attn_bwd, attn_bwd_masked and attn_bwd_noalloc. With
-// use_static the scratch rows live in g_bwd_scratch instead of `workspace`.
-attn_status bwd_impl(const void* q, const void* k, const void* v, const void* o,
-                     const float* lse, const void* dO, void* dq, void* dk, void* dv,
-                     void* workspace, size_t workspace_bytes, bool use_static, int B, int Hq,
-                     int Hkv, int Nq, int Nk, int d, float scale, int causal, int window_left,
-                     int window_right, cudaStream_t stream) {
-  g_last_error[0] = '\0';
-  bool no_rows = false, no_keys = false;
-  attn_status st = check_common(B, Hq, Hkv, Nq, Nk, d, scale, causal, &no_rows, &no_keys);
-  if (st != ATTN_OK) return st;
-  if (B == 0 || (no_rows && no_keys)) return ATTN_OK;
+// Backward shared by every backward entry point. With use_static the scratch
+// rows live in g_bwd_scratch instead of `workspace`.
+attn_status bwd_run(const void* q, const void* k, const void* v, const void* o,
+                    const float* lse, const void* dO, void* dq, void* dk, void* dv,
+                    void* workspace, size_t workspace_bytes, bool use_static, const int* cu_q,
+                    const int* cu_k, const Problem& p, const Layout& L, bool no_rows,
+                    bool no_keys, cudaStream_t stream) {
+  if (p.B == 0 || (no_rows && no_keys)) return ATTN_OK;
   const void* ptrs[10] = {q, k, v, o, lse, dO, dq, dk, dv, workspace};
   const char* names[10] = {"q", "k", "v", "o", "lse", "dO", "dq", "dk", "dv", "workspace"};
   const bool work = !no_rows && !no_keys;
   const bool used[10] = {work, work, work, work, work, work, !no_rows, !no_keys, !no_keys,
                          work && !use_static};
-  if ((st = check_args(ptrs, names, used, 10)) != ATTN_OK) return st;
-  const size_t need = attn_bwd_workspace_size(B, Hq, Nq, d);
+  const bool packed = p.geom.cu_q != nullptr || cu_q != nullptr || cu_k != nullptr;
+  attn_status st = check_args(ptrs, names, used, 10);
+  if (st != ATTN_OK) return st;
+  if (packed && (st = check_offsets_args(cu_q, cu_k)) != ATTN_OK) return st;
+  const size_t need = attn_bwd_workspace_size(p.B, p.Hq, p.geom.Nq, p.d);
   if (work && use_static && need > kStaticScratchBytes)
     return fail(ATTN_ERR_ARG,
                 "attn_bwd_noalloc: this shape needs %zu bytes of scratch, but the static area "
@@ -490,56 +594,108 @@ attn_status bwd_impl(const void* q, const void* k, const void* v, const void* o,
     return fail(ATTN_ERR_ARG, "workspace is %zu bytes, needs %zu", workspace_bytes, need);
   if ((st = ensure_init()) != ATTN_OK) return st;
   if ((st = check_used_ptrs(ptrs, names, used, 10)) != ATTN_OK) return st;
+  if (packed && (st = check_offsets(cu_q, cu_k)) != ATTN_OK) return st;
   if (!work) {
     // No keys: dQ = 0. No queries: dK = dV = 0. (The other side is empty.)
-    const size_t kv_bytes = static_cast<size_t>(B) * Hkv * Nk * d * 2;
-    const size_t q_bytes = static_cast<size_t>(B) * Hq * Nq * d * 2;
     cudaError_t e = cudaSuccess;
-    if (!no_rows) e = cudaMemsetAsync(dq, 0, q_bytes, stream);
-    if (e == cudaSuccess && !no_keys) e = cudaMemsetAsync(dk, 0, kv_bytes, stream);
-    if (e == cudaSuccess && !no_keys) e = cudaMemsetAsync(dv, 0, kv_bytes, stream);
+    if (!no_rows) e = cudaMemsetAsync(dq, 0, static_cast<size_t>(L.q_elems) * 2, stream);
+    if (e == cudaSuccess && !no_keys)
+      e = cudaMemsetAsync(dk, 0, static_cast<size_t>(L.k_elems) * 2, stream);
+    if (e == cudaSuccess && !no_keys)
+      e = cudaMemsetAsync(dv, 0, static_cast<size_t>(L.k_elems) * 2, stream);
     if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(gradients)");
     return ATTN_OK;
   }
   void* scratch = workspace;
   if (use_static && (st = static_scratch_ptr(&scratch)) != ATTN_OK) return st;
-  CUtensorMap mq, mk, mv, mdo;
-  if ((st = make_map(&mq, q, d, Nq, B * Hq)) != ATTN_OK) return st;
-  if ((st = make_map(&mk, k, d, Nk, B * Hkv)) != ATTN_OK) return st;
-  if ((st = make_map(&mv, v, d, Nk, B * Hkv)) != ATTN_OK) return st;
-  if ((st = make_map(&mdo, dO, d, Nq, B * Hq)) != ATTN_OK) return st;
+  BwdArgs a;
+  if ((st = make_map(&a.mq, q, p.d, L.q_rows, L.q_z, L.q_rs, L.q_zs)) != ATTN_OK) return st;
+  if ((st = make_map(&a.mk, k, p.d, L.k_rows, L.k_z, L.k_rs, L.k_zs)) != ATTN_OK) return st;
+  if ((st = make_map(&a.mv, v, p.d, L.k_rows, L.k_z, L.k_rs, L.k_zs)) != ATTN_OK) return st;
+  if ((st = make_map(&a.mdo, dO, p.d, L.q_rows, L.q_z, L.q_rs, L.q_zs)) != ATTN_OK) return st;
   // The preprocess kernel writes every scratch row the other two kernels
   // read, so nothing left from an earlier call is ever used and no clearing
   // is needed (this matters for the static area).
-  float* L = static_cast<float*>(scratch);
-  float* Dv = L + static_cast<size_t>(B) * Hq * attn::pad128(Nq);
-  const MaskSpec m = mask_spec(Nq, Nk, causal, window_left, window_right);
-  BwdArgs a{mq, mk, mv, mdo, o, lse, dO, dq, dk, dv, L, Dv, B, Hq, Hkv, Nq, Nk, scale, m.win};
-  if (d == 64) return dispatch_bwd<64>(a, m.mode, stream);
-  return dispatch_bwd<128>(a, m.mode, stream);
+  a.o = o; a.lse = lse; a.dO = dO; a.dq = dq; a.dk = dk; a.dv = dv;
+  a.L = static_cast<float*>(scratch);
+  a.Dv = a.L + static_cast<size_t>(p.B) * p.Hq * attn::pad128(p.geom.Nq);
+  if (p.d == 64) return dispatch_bwd<64>(a, p, stream);
+  return dispatch_bwd<128>(a, p, stream);
+}
+
+attn_status fwd_fixed(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                      int Hq, int Hkv, int Nq, int Nk, int d, float scale, int causal, int wl,
+                      int wr, float softcap, cudaStream_t stream) {
+  g_last_error[0] = '\0';
+  bool eq = false, ek = false;
+  attn_status st = check_shape(B, Hq, Hkv, Nq, d, scale, &eq);
+  if (st != ATTN_OK) return st;
+  if ((st = check_shape(B, Hq, Hkv, Nk, d, scale, &ek)) != ATTN_OK) return st;
+  if ((st = check_mask_args(causal, softcap)) != ATTN_OK) return st;
+  Problem p;
+  Layout L;
+  fixed_problem(B, Hq, Hkv, Nq, Nk, d, scale, causal, wl, wr, softcap, &p, &L);
+  return fwd_run(q, k, v, o, lse, nullptr, nullptr, p, L, eq, ek, stream);
+}
+
+attn_status bwd_fixed(const void* q, const void* k, const void* v, const void* o,
+                      const float* lse, const void* dO, void* dq, void* dk, void* dv,
+                      void* workspace, size_t workspace_bytes, bool use_static, int B, int Hq,
+                      int Hkv, int Nq, int Nk, int d, float scale, int causal, int wl, int wr,
+                      float softcap, cudaStream_t stream) {
+  g_last_error[0] = '\0';
+  bool eq = false, ek = false;
+  attn_status st = check_shape(B, Hq, Hkv, Nq, d, scale, &eq);
+  if (st != ATTN_OK) return st;
+  if ((st = check_shape(B, Hq, Hkv, Nk, d, scale, &ek)) != ATTN_OK) return st;
+  if ((st = check_mask_args(causal, softcap)) != ATTN_OK) return st;
+  Problem p;
+  Layout L;
+  fixed_problem(B, Hq, Hkv, Nq, Nk, d, scale, causal, wl, wr, softcap, &p, &L);
+  return bwd_run(q, k, v, o, lse, dO, dq, dk, dv, workspace, workspace_bytes, use_static, nullptr,
+                 nullptr, p, L, eq, ek, stream);
 }
 
 }  // namespace
 
 extern "C" {
 
-int attn_abi_version(void) { return 101; }
+int attn_abi_version(void) { return 102; }
 
 const char* attn_get_last_error(void) { return g_last_error; }
 
 attn_status attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B,
                      int Hq, int Hkv, int N, int d, float scale, int causal,
                      attn_stream_t stream_) {
-  return fwd_impl(q, k, v, o, lse, B, Hq, Hkv, N, N, d, scale, causal, -1, -1,
-                  static_cast<cudaStream_t>(stream_));
+  return fwd_fixed(q, k, v, o, lse, B, Hq, Hkv, N, N, d, scale, causal, -1, -1, 0.f,
+                   static_cast<cudaStream_t>(stream_));
 }
 
 attn_status attn_fwd_masked(const void* q, const void* k, const void* v, void* o, float* lse,
                             int B, int Hq, int Hkv, int Nq, int Nk, int d, float scale,
-                            int causal, int window_left, int window_right,
+                            int causal, int window_left, int window_right, float softcap,
                             attn_stream_t stream_) {
-  return fwd_impl(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, scale, causal, window_left,
-                  window_right, static_cast<cudaStream_t>(stream_));
+  return fwd_fixed(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, scale, causal, window_left,
+                   window_right, softcap, static_cast<cudaStream_t>(stream_));
+}
+
+attn_status attn_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* lse,
+                            const int* cu_seqlens_q, const int* cu_seqlens_k, int B, int Hq,
+                            int Hkv, int total_q, int total_k, int max_seqlen_q,
+                            int max_seqlen_k, int d, float scale, int causal, int window_left,
+                            int window_right, float softcap, attn_stream_t stream_) {
+  g_last_error[0] = '\0';
+  bool no_rows = false, no_keys = false;
+  attn_status st = check_packed(B, Hq, Hkv, total_q, total_k, max_seqlen_q, max_seqlen_k, d,
+                                scale, &no_rows, &no_keys);
+  if (st != ATTN_OK) return st;
+  if ((st = check_mask_args(causal, softcap)) != ATTN_OK) return st;
+  Problem p;
+  Layout L;
+  packed_problem(cu_seqlens_q, cu_seqlens_k, B, Hq, Hkv, total_q, total_k, max_seqlen_q,
+                 max_seqlen_k, d, scale, causal, window_left, window_right, softcap, &p, &L);
+  return fwd_run(q, k, v, o, lse, cu_seqlens_q, cu_seqlens_k, p, L, no_rows, no_keys,
+                 static_cast<cudaStream_t>(stream_));
 }
 
 size_t attn_bwd_workspace_size(int B, int Hq, int N, int d) {
@@ -554,27 +710,49 @@ attn_status attn_bwd(const void* q, const void* k, const void* v, const void* o,
                      const float* lse, const void* dO, void* dq, void* dk, void* dv,
                      void* workspace, size_t workspace_bytes, int B, int Hq, int Hkv, int N,
                      int d, float scale, int causal, attn_stream_t stream_) {
-  return bwd_impl(q, k, v, o, lse, dO, dq, dk, dv, workspace, workspace_bytes, false, B, Hq, Hkv,
-                  N, N, d, scale, causal, -1, -1, static_cast<cudaStream_t>(stream_));
+  return bwd_fixed(q, k, v, o, lse, dO, dq, dk, dv, workspace, workspace_bytes, false, B, Hq, Hkv,
+                   N, N, d, scale, causal, -1, -1, 0.f, static_cast<cudaStream_t>(stream_));
 }
 
 attn_status attn_bwd_masked(const void* q, const void* k, const void* v, const void* o,
                             const float* lse, const void* dO, void* dq, void* dk, void* dv,
                             void* workspace, size_t workspace_bytes, int B, int Hq, int Hkv,
                             int Nq, int Nk, int d, float scale, int causal, int window_left,
-                            int window_right, attn_stream_t stream_) {
-  return bwd_impl(q, k, v, o, lse, dO, dq, dk, dv, workspace, workspace_bytes, false, B, Hq, Hkv,
-                  Nq, Nk, d, scale, causal, window_left, window_right,
-                  static_cast<cudaStream_t>(stream_));
+                            int window_right, float softcap, attn_stream_t stream_) {
+  return bwd_fixed(q, k, v, o, lse, dO, dq, dk, dv, workspace, workspace_bytes, false, B, Hq, Hkv,
+                   Nq, Nk, d, scale, causal, window_left, window_right, softcap,
+                   static_cast<cudaStream_t>(stream_));
+}
+
+attn_status attn_bwd_varlen(const void* q, const void* k, const void* v, const void* o,
+                            const float* lse, const void* dO, void* dq, void* dk, void* dv,
+                            const int* cu_seqlens_q, const int* cu_seqlens_k, void* workspace,
+                            size_t workspace_bytes, int B, int Hq, int Hkv, int total_q,
+                            int total_k, int max_seqlen_q, int max_seqlen_k, int d, float scale,
+                            int causal, int window_left, int window_right, float softcap,
+                            attn_stream_t stream_) {
+  g_last_error[0] = '\0';
+  bool no_rows = false, no_keys = false;
+  attn_status st = check_packed(B, Hq, Hkv, total_q, total_k, max_seqlen_q, max_seqlen_k, d,
+                                scale, &no_rows, &no_keys);
+  if (st != ATTN_OK) return st;
+  if ((st = check_mask_args(causal, softcap)) != ATTN_OK) return st;
+  Problem p;
+  Layout L;
+  packed_problem(cu_seqlens_q, cu_seqlens_k, B, Hq, Hkv, total_q, total_k, max_seqlen_q,
+                 max_seqlen_k, d, scale, causal, window_left, window_right, softcap, &p, &L);
+  return bwd_run(q, k, v, o, lse, dO, dq, dk, dv, workspace, workspace_bytes, false, cu_seqlens_q,
+                 cu_seqlens_k, p, L, no_rows, no_keys, static_cast<cudaStream_t>(stream_));
 }
 
 attn_status attn_bwd_noalloc(const void* q, const void* k, const void* v, const void* o,
                              const float* lse, const void* dO, void* dq, void* dk, void* dv,
                              int B, int Hq, int Hkv, int N, int d, float scale, int causal,
                              attn_stream_t stream_) {
-  return bwd_impl(q, k, v, o, lse, dO, dq, dk, dv, nullptr, 0, true, B, Hq, Hkv, N, N, d, scale,
-                  causal, -1, -1, static_cast<cudaStream_t>(stream_));
+  return bwd_fixed(q, k, v, o, lse, dO, dq, dk, dv, nullptr, 0, true, B, Hq, Hkv, N, N, d, scale,
+                   causal, -1, -1, 0.f, static_cast<cudaStream_t>(stream_));
 }
+
 
 attn_status attn_selftest_wait_timeout(attn_stream_t stream_) {
   g_last_error[0] = '\0';
@@ -639,6 +817,10 @@ attn_status attn_check_status(attn_stream_t stream_) {
     const int zero = 0;
     e = cudaMemcpyToSymbol(attn::g_attn_device_status, &zero, sizeof(int));
     if (e != cudaSuccess) return cuda_fail(e, "clear status word");
+    if ((word & 0xFF) == attn::kDevBadOffsets)
+      return fail(ATTN_ERR_ARG,
+                  "cu_seqlens offsets out of range (negative, decreasing, past the packed "
+                  "tensor, or a sequence longer than max_seqlen); they were clipped");
     return fail(ATTN_ERR_TIMEOUT, "kernel gave up on a pipeline wait (code %d, site %d)",
                 word & 0xFF, (word >> 8) & 0xFF);
   }

@@ -33,6 +33,7 @@
 // 64*(kk/4) + 8*(kk%4) of the tile.
 #pragma once
 
+#include "geometry.cuh"
 #include "sm100.cuh"
 #include "visibility.cuh"
 
@@ -44,21 +45,28 @@ __host__ __device__ inline int pad128(int n) { return (n + 127) & ~127; }
 
 // ------------------------------------------------------------------ preprocess
 // 8 lanes per query row, 4 rows per warp, 32 rows per 256-thread block. The
-// grid covers BH * Npad rows exactly (a multiple of 128), so every shuffle
-// group is fully populated.
+// grid covers B * Hq * Npad workspace rows exactly (Npad a multiple of 128),
+// so every shuffle group is fully populated. Workspace row (b * Hq + h) * Npad
+// + n holds query n of sequence b, head h; rows past the sequence get
+// -lse*log2(e) = -inf (so P = 0 there) and D = 0.
 template <int D>
 __global__ void __launch_bounds__(256)
 bwd_pre_kernel(const __nv_bfloat16* __restrict__ o, const __nv_bfloat16* __restrict__ dO,
-               const float* __restrict__ lse, float* __restrict__ L, float* __restrict__ Dv, int N,
-               int Npad) {
+               const float* __restrict__ lse, float* __restrict__ L, float* __restrict__ Dv,
+               int Hq, SeqGeom geom, int Npad) {
   const long long row = static_cast<long long>(blockIdx.x) * 32 + (threadIdx.x >> 3);
   const int sub = threadIdx.x & 7;
   const long long bh = row / Npad;
   const int n = static_cast<int>(row - bh * Npad);
+  const int b = static_cast<int>(bh / Hq);
+  const int h = static_cast<int>(bh - static_cast<long long>(b) * Hq);
+  const SeqSpan sp = geom.cu_q ? seq_span<true>(geom, b) : seq_span<false>(geom, b);
+  const long long z = geom.cu_q ? h : bh;
+  const int N = sp.nq;
   float acc = 0.f;
   if (n < N) {
     constexpr int kPer = D / 8;  // elements per lane: 16 (D=128) or 8 (D=64)
-    const size_t base = (static_cast<size_t>(bh) * N + n) * D + sub * kPer;
+    const size_t base = z * geom.o_z + (sp.q0 + n) * geom.o_row + sub * kPer;
     const uint4* po = reinterpret_cast<const uint4*>(o + base);
     const uint4* pd = reinterpret_cast<const uint4*>(dO + base);
 #pragma unroll
@@ -76,7 +84,7 @@ bwd_pre_kernel(const __nv_bfloat16* __restrict__ o, const __nv_bfloat16* __restr
   acc += __shfl_xor_sync(0xffffffffu, acc, 2);
   acc += __shfl_xor_sync(0xffffffffu, acc, 1);
   if (sub == 0) {
-    const float l = (n < N) ? lse[static_cast<size_t>(bh) * N + n] : -INFINITY;
+    const float l = (n < N) ? lse[z * geom.lse_z + sp.q0 + n] : -INFINITY;
     // A row that saw no key (lse = -inf) is treated like padding: P = 0.
     L[row] = (l == -INFINITY) ? -INFINITY : -l * kLog2e;
     Dv[row] = (n < N) ? -acc : 0.f;
@@ -160,13 +168,17 @@ struct DkdvCfg {
   static constexpr int kThreads = 384;
 };
 
-template <int D, int MODE>
+template <int D, int MODE, int FEAT>
 __global__ void __launch_bounds__(384, 1)
 bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
                 const float* __restrict__ Lws, const float* __restrict__ Dws,
                 __nv_bfloat16* __restrict__ dk, __nv_bfloat16* __restrict__ dv, int Hq, int group,
-                int Nq, int Nk, int Npad, float scale_log2, float scale, KeyWindow win) {
+                SeqGeom geom, int Npad, float scale_log2, float scale, KeyWindow win,
+                Softcap cap) {
+  constexpr bool SOFTCAP = (FEAT & kFeatSoftcap) != 0;
+  constexpr bool PACKED = (FEAT & kFeatPacked) != 0;
+  static_assert(FEAT == 0 || MODE == kMaskGeneral, "features run in the general mode");
   using C = DkdvCfg<D>;
   constexpr int NS = C::kStages;
   extern __shared__ uint8_t smem_raw[];
@@ -190,11 +202,16 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   // 1-D grid, KV block fastest, then (batch, KV head): CTAs resident
   // together mostly share one head's Q/dO in L2. Low j has the most causal
   // work and launches first within its head.
-  const int nkv = (Nk + 127) >> 7;
+  const int nkv = (geom.Nk + 127) >> 7;
   const int bh_kv = blockIdx.x / nkv;
   const int b = bh_kv / Hkv;
   const int hkv = bh_kv - b * Hkv;
   const int j = blockIdx.x - bh_kv * nkv;
+  const SeqSpan sp = seq_span<PACKED>(geom, b);
+  const int Nq = sp.nq, Nk = sp.nk;
+  if (j * 128 >= Nk) return;                  // packed batch: past this sequence's keys
+  win.off = Nk - Nq;                          // bottom-right alignment per sequence
+  const int zkv = PACKED ? hkv : bh_kv;       // TMA z of this KV head
   int i_start, i_end;                         // query blocks that see key tile j
   q_block_range<MODE>(j, Nq, Nk, win, i_start, i_end);
   const int per_head = max(0, i_end - i_start + 1);
@@ -241,8 +258,8 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         mbar_expect_tx(kv_full, 2 * C::kTile);
 #pragma unroll
         for (int a = 0; a < D / 64; ++a) {
-          tma_load_3d(smem + C::kKOff + a * 16384, &tm_k, kv_full, a * 64, j * 128, bh_kv);
-          tma_load_3d(smem + C::kVOff + a * 16384, &tm_v, kv_full, a * 64, j * 128, bh_kv);
+          tma_load_3d(smem + C::kKOff + a * 16384, &tm_k, kv_full, a * 64, sp.k0 + j * 128, zkv);
+          tma_load_3d(smem + C::kVOff + a * 16384, &tm_v, kv_full, a * 64, sp.k0 + j * 128, zkv);
         }
       }
       int issued = 0;
@@ -251,12 +268,14 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         if (round > 0 && !mbar_wait(&ld_empty[st], (round - 1) & 1, abort_flag, kSiteBLoadEmpty)) break;
         int i, bh_q;
         step_head(s, i, bh_q);
+        const int zq = PACKED ? bh_q - b * Hq : bh_q;
         uint8_t* stage = smem + C::kStageOff + st * C::kStageBytes;
         mbar_expect_tx(&ld_full[st], 2 * C::kTile + 1024);
 #pragma unroll
         for (int a = 0; a < D / 64; ++a) {
-          tma_load_3d(stage + a * 16384, &tm_q, &ld_full[st], a * 64, i * 128, bh_q);
-          tma_load_3d(stage + C::kTile + a * 16384, &tm_do, &ld_full[st], a * 64, i * 128, bh_q);
+          tma_load_3d(stage + a * 16384, &tm_q, &ld_full[st], a * 64, sp.q0 + i * 128, zq);
+          tma_load_3d(stage + C::kTile + a * 16384, &tm_do, &ld_full[st], a * 64,
+                      sp.q0 + i * 128, zq);
         }
         const size_t off = static_cast<size_t>(bh_q) * Npad + i * 128;
         bulk_load(stage + 2 * C::kTile, Lws + off, 512, &ld_full[st]);
@@ -376,9 +395,20 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         for (int e = 0; e < 16; ++e) {
           const int c = c_base + c0 + 2 * e;
           const float2 nl = *reinterpret_cast<const float2*>(&Ls[c0 + 2 * e]);
-          const float2 x = ffma2(make_float2(u2f(r[2 * e]), u2f(r[2 * e + 1])), sc2, nl);
-          float p0 = fast_exp2(x.x);
-          float p1 = fast_exp2(x.y);
+          float p0, p1, g0 = 1.f, g1 = 1.f;
+          if constexpr (SOFTCAP) {
+            // P from the capped logit; dS gets the chain-rule factor 1 - t^2.
+            const float t0 = softcap_tanh(u2f(r[2 * e]), cap);
+            const float t1 = softcap_tanh(u2f(r[2 * e + 1]), cap);
+            p0 = fast_exp2(fmaf(cap.out, t0, nl.x));
+            p1 = fast_exp2(fmaf(cap.out, t1, nl.y));
+            g0 = fmaf(-t0, t0, 1.f);
+            g1 = fmaf(-t1, t1, 1.f);
+          } else {
+            const float2 x = ffma2(make_float2(u2f(r[2 * e]), u2f(r[2 * e + 1])), sc2, nl);
+            p0 = fast_exp2(x.x);
+            p1 = fast_exp2(x.y);
+          }
           if (edge) {
             if (MODE == kMaskGeneral) {
               if (c < c_lo || c > c_hi) p0 = 0.f;
@@ -388,8 +418,8 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
               if (c + 1 < c_lo) p1 = 0.f;
             }
           }
-          pf[c0 + 2 * e] = p0;
-          pf[c0 + 2 * e + 1] = p1;
+          pf[c0 + 2 * e] = SOFTCAP ? p0 * g0 : p0;
+          pf[c0 + 2 * e + 1] = SOFTCAP ? p1 * g1 : p1;
           pw[c0 / 2 + e] = pack_bf16x2(p0, p1);
         }
       };
@@ -422,7 +452,9 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     if (ok && n_steps > 0) ok = mbar_wait(acc_done, 0, abort_flag, kSiteBAcc);
     if (ok) {
       const bool valid = key < Nk;
-      const size_t row_off = (static_cast<size_t>(bh_kv) * Nk + (valid ? key : 0)) * D;
+      const long long kv_z = PACKED ? geom.kv_z : static_cast<long long>(Nk) * D;
+      const long long kv_row = PACKED ? geom.kv_row : D;
+      const size_t row_off = zkv * kv_z + (sp.k0 + (valid ? key : 0)) * kv_row;
       if (n_steps > 0) {
         tc_fence_after();
         if (h == 0)
@@ -463,13 +495,16 @@ struct DqCfg {
   static constexpr int kThreads = 384;
 };
 
-template <int D, int MODE>
+template <int D, int MODE, int FEAT>
 __global__ void __launch_bounds__(384, 1)
 bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
               const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
               const float* __restrict__ Lws, const float* __restrict__ Dws,
-              __nv_bfloat16* __restrict__ dq, int Hq, int group, int Nq, int Nk, int Npad,
-              float scale_log2, float scale, KeyWindow win) {
+              __nv_bfloat16* __restrict__ dq, int Hq, int group, SeqGeom geom, int Npad,
+              float scale_log2, float scale, KeyWindow win, Softcap cap) {
+  constexpr bool SOFTCAP = (FEAT & kFeatSoftcap) != 0;
+  constexpr bool PACKED = (FEAT & kFeatPacked) != 0;
+  static_assert(FEAT == 0 || MODE == kMaskGeneral, "features run in the general mode");
   using C = DqCfg<D>;
   constexpr int NS = C::kStages;
   extern __shared__ uint8_t smem_raw[];
@@ -491,13 +526,17 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
   const int warp = warp_id(), lane = lane_id();
   // 1-D grid, query block fastest (heaviest causal block first), then
   // (batch, query head): CTAs resident together mostly share one head's K/V.
-  const int nqb = (Nq + 127) >> 7;
-  const int nkv = (Nk + 127) >> 7;
+  const int nqb = (geom.Nq + 127) >> 7;
   const int bh = blockIdx.x / nqb;
   const int b = bh / Hq;
   const int hq = bh - b * Hq;
-  const int bh_kv = b * (Hq / group) + hq / group;
   const int i = nqb - 1 - (blockIdx.x - bh * nqb);
+  const SeqSpan sp = seq_span<PACKED>(geom, b);
+  const int Nq = sp.nq, Nk = sp.nk;
+  if (i * 128 >= Nq) return;                 // packed batch: past this sequence's rows
+  win.off = Nk - Nq;                         // bottom-right alignment per sequence
+  const int zq = PACKED ? hq : bh;           // TMA z of the query head and its KV head
+  const int zkv = PACKED ? hq / group : b * (Hq / group) + hq / group;
   int j_lo, j_hi;                            // key tiles this query block sees
   kv_tile_range<MODE>(i * 128, min(i * 128 + 127, Nq - 1), Nk, win, j_lo, j_hi);
   const int n = max(0, j_hi - j_lo + 1);
@@ -537,8 +576,8 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         mbar_expect_tx(qd_full, 2 * C::kTile);
 #pragma unroll
         for (int a = 0; a < D / 64; ++a) {
-          tma_load_3d(smem + C::kQOff + a * 16384, &tm_q, qd_full, a * 64, i * 128, bh);
-          tma_load_3d(smem + C::kDOOff + a * 16384, &tm_do, qd_full, a * 64, i * 128, bh);
+          tma_load_3d(smem + C::kQOff + a * 16384, &tm_q, qd_full, a * 64, sp.q0 + i * 128, zq);
+          tma_load_3d(smem + C::kDOOff + a * 16384, &tm_do, qd_full, a * 64, sp.q0 + i * 128, zq);
         }
       }
       uint32_t issued = 0;
@@ -554,7 +593,7 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
 #pragma unroll
           for (int a = 0; a < D / 64; ++a)
             tma_load_3d(smem + C::kKVOff + s * C::kTile + a * 16384, w ? &tm_v : &tm_k, &kv_full[s],
-                        a * 64, (j_lo + jj) * 128, bh_kv);
+                        a * 64, sp.k0 + (j_lo + jj) * 128, zkv);
           ++issued;
         }
       }
@@ -671,9 +710,18 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
           const int c = c_base + c0 + 2 * e;
-          const float2 x = ffma2(make_float2(u2f(r[2 * e]), u2f(r[2 * e + 1])), sc2, nl2);
-          float p0 = fast_exp2(x.x);
-          float p1 = fast_exp2(x.y);
+          float p0, p1;
+          if constexpr (SOFTCAP) {
+            // dS needs P * (1 - t^2): the chain rule through c * tanh(z / c).
+            const float t0 = softcap_tanh(u2f(r[2 * e]), cap);
+            const float t1 = softcap_tanh(u2f(r[2 * e + 1]), cap);
+            p0 = fast_exp2(fmaf(cap.out, t0, nLr)) * fmaf(-t0, t0, 1.f);
+            p1 = fast_exp2(fmaf(cap.out, t1, nLr)) * fmaf(-t1, t1, 1.f);
+          } else {
+            const float2 x = ffma2(make_float2(u2f(r[2 * e]), u2f(r[2 * e + 1])), sc2, nl2);
+            p0 = fast_exp2(x.x);
+            p1 = fast_exp2(x.y);
+          }
           if (edge) {
             if (MODE == kMaskGeneral) {
               if (c < c_lo || c > c_hi) p0 = 0.f;
@@ -711,7 +759,9 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     if (ok && n > 0) ok = mbar_wait(acc_done, 0, abort_flag, kSiteBAcc);
     if (ok) {
       const bool valid = row < Nq;
-      __nv_bfloat16* dst = dq + (static_cast<size_t>(bh) * Nq + (valid ? row : 0)) * D;
+      const long long o_z = PACKED ? geom.o_z : static_cast<long long>(Nq) * D;
+      const long long o_row = PACKED ? geom.o_row : D;
+      __nv_bfloat16* dst = dq + zq * o_z + (sp.q0 + (valid ? row : 0)) * o_row;
       if (n > 0) {
         tc_fence_after();
         if (h == 0)

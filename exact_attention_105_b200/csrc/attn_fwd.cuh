@@ -37,6 +37,7 @@
 // the MN-major SW128 layout for V.
 #pragma once
 
+#include "geometry.cuh"
 #include "sm100.cuh"
 #include "visibility.cuh"
 
@@ -75,12 +76,15 @@ constexpr int kFwdRegsSoftmax = 216;
 constexpr int kFwdRegsSmall = 72;
 static_assert(2 * kFwdRegsSoftmax + kFwdRegsSmall <= 3 * kFwdRegsLaunch, "register split");
 
-template <int D, int MODE>
+template <int D, int MODE, int FEAT>
 __global__ void __launch_bounds__(384, 1)
 fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
            const __grid_constant__ CUtensorMap tm_v, __nv_bfloat16* __restrict__ out,
-           float* __restrict__ lse_out, int Hq, int group, int Nq, int Nk, float scale_log2,
-           KeyWindow win) {
+           float* __restrict__ lse_out, int Hq, int group, SeqGeom geom, float scale_log2,
+           KeyWindow win, Softcap cap) {
+  constexpr bool SOFTCAP = (FEAT & kFeatSoftcap) != 0;
+  constexpr bool PACKED = (FEAT & kFeatPacked) != 0;
+  static_assert(FEAT == 0 || MODE == kMaskGeneral, "features run in the general mode");
   using C = FwdCfg<D>;
   constexpr int NS = C::kStages;
   extern __shared__ uint8_t smem_raw[];
@@ -103,33 +107,38 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
   // 1-D grid, (batch, query head) fastest, then 256-row query block from the
   // last (heaviest when causal) to the first: every head's heaviest block is
   // dispatched before any lighter one, which keeps the causal tail short.
-  const int nmb = (Nq + 255) >> 8;
+  const int nmb = (geom.Nq + 255) >> 8;
   const int BH = gridDim.x / nmb;
   const int bh = blockIdx.x % BH;                  // b * Hq + hq
   const int b = bh / Hq;
   const int hq = bh - b * Hq;
-  const int bh_kv = b * (Hq / group) + hq / group; // GQA: contiguous head groups
   const int mb = nmb - 1 - static_cast<int>(blockIdx.x / BH);
+  const SeqSpan sp = seq_span<PACKED>(geom, b);
+  const int Nq = sp.nq, Nk = sp.nk;
+  if (mb * 256 >= Nq) return;                      // packed batch: past this sequence's rows
+  win.off = Nk - Nq;                               // bottom-right alignment per sequence
+  // TMA z coordinates of the query head and its KV head (GQA: contiguous groups).
+  const int zq = PACKED ? hq : bh;
+  const int zkv = PACKED ? hq / group : b * (Hq / group) + hq / group;
   const int nkv = (Nk + 127) >> 7;
 
-  // Per query tile t: KV tiles [lo_t[t], hi_t[t]] (n_t[t] of them). A tile whose
+  // Per query tile t: KV tiles [lo_t(t), hi_t(t)] (n_t(t) of them). A tile whose
   // rows exist but see no key has n_t = 0 and writes O = 0, lse = -inf. The
-  // CTA streams KV tiles jb..je, the union of its tiles' ranges.
-  int lo_t[2], hi_t[2], n_t[2];
-#pragma unroll
-  for (int t = 0; t < 2; ++t) {
-    const int r0 = mb * 256 + t * 128;
-    if (r0 >= Nq) {
-      lo_t[t] = 0;
-      hi_t[t] = -1;
-    } else {
-      kv_tile_range<MODE>(r0, min(r0 + 127, Nq - 1), Nk, win, lo_t[t], hi_t[t]);
-    }
-    n_t[t] = max(0, hi_t[t] - lo_t[t] + 1);
-  }
-  const int jb = (n_t[0] > 0) ? lo_t[0] : lo_t[1];
-  const int je = (n_t[1] > 0) ? hi_t[1] : hi_t[0];
-  const int n_span = (n_t[0] > 0 || n_t[1] > 0) ? je - jb + 1 : 0;
+  // CTA streams KV tiles jb..je, the union of its tiles' ranges. The bounds
+  // are scalars with select accessors, never an array indexed by a runtime
+  // tile number: that would live in local memory and be reloaded after every
+  // barrier wait on the MMA issue path.
+  int lo0 = 0, hi0 = -1, lo1 = 0, hi1 = -1;
+  if (mb * 256 < Nq) kv_tile_range<MODE>(mb * 256, min(mb * 256 + 127, Nq - 1), Nk, win, lo0, hi0);
+  if (mb * 256 + 128 < Nq)
+    kv_tile_range<MODE>(mb * 256 + 128, min(mb * 256 + 255, Nq - 1), Nk, win, lo1, hi1);
+  const int n0 = max(0, hi0 - lo0 + 1), n1 = max(0, hi1 - lo1 + 1);
+  auto lo_t = [&](int t) { return t ? lo1 : lo0; };
+  auto hi_t = [&](int t) { return t ? hi1 : hi0; };
+  auto n_t = [&](int t) { return t ? n1 : n0; };
+  const int jb = (n_t(0) > 0) ? lo_t(0) : lo_t(1);
+  const int je = (n_t(1) > 0) ? hi_t(1) : hi_t(0);
+  const int n_span = (n_t(0) > 0 || n_t(1) > 0) ? je - jb + 1 : 0;
 
   if (threadIdx.x == 0) {
     mbar_init(&q_full[0], 1);
@@ -165,12 +174,12 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
       tma_prefetch_desc(&tm_v);
 #pragma unroll
       for (int t = 0; t < 2; ++t) {
-        if (n_t[t] > 0) {
+        if (n_t(t) > 0) {
           mbar_expect_tx(&q_full[t], C::kTxBytes);
 #pragma unroll
           for (int a = 0; a < D / 64; ++a)
             tma_load_3d(smem + C::kQOff + t * C::kTileBytes + a * 16384, &tm_q, &q_full[t],
-                        a * 64, mb * 256 + t * 128, bh);
+                        a * 64, sp.q0 + mb * 256 + t * 128, zq);
         }
       }
       uint32_t issued = 0;
@@ -187,14 +196,14 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
 #pragma unroll
           for (int a = 0; a < D / 64; ++a)
             tma_load_3d(smem + C::kKVOff + s * C::kTileBytes + a * 16384, w ? &tm_v : &tm_k,
-                        &kv_full[s], a * 64, j * 128, bh_kv);
+                        &kv_full[s], a * 64, sp.k0 + j * 128, zkv);
           ++issued;
         }
       }
       // Let every copy this thread started land before the CTA can exit.
 #pragma unroll
       for (int t = 0; t < 2; ++t)
-        if (n_t[t] > 0) mbar_wait_drain(&q_full[t], 0);
+        if (n_t(t) > 0) mbar_wait_drain(&q_full[t], 0);
       const uint32_t first = issued > (uint32_t)NS ? issued - NS : 0u;
       for (uint32_t i = first; i < issued; ++i) mbar_wait_drain(&kv_full[i % NS], (i / NS) & 1u);
     } else if (warp == 9 && lane == 0) {
@@ -225,14 +234,14 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
       bool ok = true;
 #pragma unroll
       for (int t = 0; t < 2; ++t)
-        if (ok && n_t[t] > 0) ok = mbar_wait(&q_full[t], 0, abort_flag, kSiteQFull);
+        if (ok && n_t(t) > 0) ok = mbar_wait(&q_full[t], 0, abort_flag, kSiteQFull);
       // Ring positions: K_j at 2 (j - jb), V_j at 2 (j - jb) + 1.
       if (ok && n_span > 0) ok = kv_wait(0);
       if (ok && n_span > 0) {
         tc_fence_after();
 #pragma unroll
         for (int t = 0; t < 2; ++t)
-          if (n_t[t] > 0 && lo_t[t] == jb) {
+          if (n_t(t) > 0 && lo_t(t) == jb) {
             issue_qk(t, 0);
             tc_commit(&s_full[t]);
           }
@@ -253,19 +262,19 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
         };
 #pragma unroll
         for (int t = 0; t < 2; ++t) {
-          if (n_t[t] == 0) continue;
-          if (j >= lo_t[t] && j <= hi_t[t]) {
-            if (!mbar_wait(&p_full[t], (j - lo_t[t]) & 1, abort_flag, kSitePFull)) { ok = false; break; }
+          if (n_t(t) == 0) continue;
+          if (j >= lo_t(t) && j <= hi_t(t)) {
+            if (!mbar_wait(&p_full[t], (j - lo_t(t)) & 1, abort_flag, kSitePFull)) { ok = false; break; }
             tc_fence_after();
-            issue_pv(t, iv % NS, j > lo_t[t]);
-            if (j == hi_t[t]) {
+            issue_pv(t, iv % NS, j > lo_t(t));
+            if (j == hi_t(t)) {
               tc_commit(&o_full[t]);
             } else {
               if (!need_k_next()) { ok = false; break; }
               issue_qk(t, ik % NS);
               tc_commit(&s_full[t]);
             }
-          } else if (lo_t[t] == j + 1) {
+          } else if (lo_t(t) == j + 1) {
             // This tile's first key tile is the next one.
             if (!need_k_next()) { ok = false; break; }
             issue_qk(t, ik % NS);
@@ -296,7 +305,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
     const uint32_t t_s = tmem + lane_base + t * 128;
     const uint32_t t_p = t_s + 64;
     const uint32_t t_o = tmem + lane_base + 256 + t * 128;
-    const int n = n_t[t];
+    const int n = n_t(t);
     const int r_first = mb * 256 + t * 128;                  // first and last row of this tile
     const int r_last = min(r_first + 127, Nq - 1);
     // Visible keys of this row: [k_lo, k_hi] (k_hi < k_lo: none).
@@ -310,7 +319,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
     float l_mma = 0.f;         // running sum of the bf16-rounded P fed to the MMA (for O)
     bool ok = n > 0;
     for (int jj = 0; ok && jj < n; ++jj) {
-      const int j = lo_t[t] + jj;                            // key tile
+      const int j = lo_t(t) + jj;                            // key tile
       const int kb = j * 128;
       if (!mbar_wait(&s_full[t], jj & 1, abort_flag, kSiteSFull)) { ok = false; break; }
       tc_fence_after();
@@ -324,6 +333,19 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
       reg_fence(r2);
       reg_fence(r3);
 
+      if constexpr (SOFTCAP) {
+        // Scores become capped logits in log2 units, in place. The mask below
+        // then sets -inf on the capped values.
+        auto cap_block = [&](uint32_t (&rr)[32]) {
+#pragma unroll
+          for (int e = 0; e < 32; ++e)
+            rr[e] = f2u(cap.out * softcap_tanh(u2f(rr[e]), cap));
+        };
+        cap_block(r0);
+        cap_block(r1);
+        cap_block(r2);
+        cap_block(r3);
+      }
       // Only tiles that straddle an edge of some row's visible range are masked.
       bool edge;
       if (MODE == kMaskNone) edge = ragged && j == nkv - 1;
@@ -358,7 +380,8 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
         mx2 = fmax3f(mx2, u2f(r2[e]), u2f(r2[e + 1]));
         mx3 = fmax3f(mx3, u2f(r3[e]), u2f(r3[e + 1]));
       }
-      const float m_tile = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * scale_log2;
+      // (Capped logits are already scaled to log2 units.)
+      const float m_tile = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * (SOFTCAP ? 1.0f : scale_log2);
       const float m_new = fmaxf(m_run, m_tile);
       // Lazy rescale: keep the stale max unless the new one is more than 2^8 larger.
       const bool need = m_new > m_run + 8.0f;
@@ -380,7 +403,8 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
         l_mma *= f;
         m_run = m_new;
       }
-      const float2 sc2 = make_float2(scale_log2, scale_log2);
+      const float sl = SOFTCAP ? 1.0f : scale_log2;
+      const float2 sc2 = make_float2(sl, sl);
       // A row with no visible key so far keeps m_run = -inf; its p are all 0.
       const float neg_m = (m_run == -INFINITY) ? 0.0f : -m_run;
       const float2 nm2 = make_float2(neg_m, neg_m);
@@ -430,7 +454,9 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
       const bool has_o = n > 0;
       if (has_o) tc_fence_after();
       const float inv_l = (l_mma > 0.f) ? 1.0f / l_mma : 0.f;
-      __nv_bfloat16* orow = out + (static_cast<size_t>(bh) * Nq + (row < Nq ? row : 0)) * D;
+      const long long o_z = PACKED ? geom.o_z : static_cast<long long>(Nq) * D;
+      const long long o_row = PACKED ? geom.o_row : D;
+      __nv_bfloat16* orow = out + zq * o_z + (sp.q0 + (row < Nq ? row : 0)) * o_row;
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
         uint32_t o[32];
@@ -453,7 +479,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
         }
       }
       if (row < Nq)
-        lse_out[static_cast<size_t>(bh) * Nq + row] =
+        lse_out[zq * (PACKED ? geom.lse_z : static_cast<long long>(Nq)) + sp.q0 + row] =
             (l_run > 0.f) ? (m_run + __log2f(l_run)) * 0.69314718055994531f : -INFINITY;
     }
   }

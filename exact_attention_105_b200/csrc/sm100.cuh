@@ -20,6 +20,7 @@ namespace attn {
 enum : int {
   kDevOk = 0,
   kDevTimeout = 1,   // low 8 bits: code; bits 8..15: which wait site gave up
+  kDevBadOffsets = 2,  // packed-batch offsets were out of range and were clipped
 };
 
 // Defined once per binary: every kernel of the library is built in one

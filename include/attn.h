@@ -43,7 +43,8 @@
  *    return ATTN_ERR_CUDA.
  *  - Kernel waits are bounded. A kernel that stalls for two seconds on a
  *    pipeline barrier records a timeout in a device status word and exits.
- *    attn_check_status() reports it.
+ *    attn_check_status() reports it (ATTN_ERR_TIMEOUT), as it reports
+ *    invalid packed-batch offsets found on the GPU (ATTN_ERR_ARG).
  */
 #ifndef EXACT_ATTENTION_B200_ATTN_H_
 #define EXACT_ATTENTION_B200_ATTN_H_
@@ -147,11 +148,16 @@ attn_status attn_bwd_noalloc(const void* q, const void* k, const void* v, const 
  *   A query row that sees no key (Nq > Nk with causal, or a window that
  *   falls outside the keys) gets o = 0 and lse = -inf. Nk == 0 with Nq > 0
  *   is such a case for every row. Nq == 0 or B == 0 writes nothing.
+ *   softcap: 0 turns it off. With softcap = c > 0 each scaled logit
+ *   z = scale * q_i . k_j becomes c * tanh(z / c) before the mask and the
+ *   softmax (release 2.6 on the same page, "softcapping as used in Gemma-2
+ *   and Grok"; the pages give no formula, this is the form those models
+ *   use), and lse is over the capped logits. Must be finite and >= 0.
  * Errors as in attn_fwd.
  */
 attn_status attn_fwd_masked(const void* q, const void* k, const void* v, void* o, float* lse,
                             int B, int Hq, int Hkv, int Nq, int Nk, int d, float scale,
-                            int causal, int window_left, int window_right,
+                            int causal, int window_left, int window_right, float softcap,
                             attn_stream_t stream);
 
 /*
@@ -168,12 +174,50 @@ attn_status attn_bwd_masked(const void* q, const void* k, const void* v, const v
                             const float* lse, const void* dO, void* dq, void* dk, void* dv,
                             void* workspace, size_t workspace_bytes, int B, int Hq, int Hkv,
                             int Nq, int Nk, int d, float scale, int causal, int window_left,
-                            int window_right, attn_stream_t stream);
+                            int window_right, float softcap, attn_stream_t stream);
+
+/*
+ * attn_fwd_varlen / attn_bwd_varlen: a packed ("varlen", release 2.0 on the
+ * same page) batch of B sequences of different lengths, stored token by
+ * token with no padding:
+ *   q, o, dO, dq [total_q, Hq, d] bf16; k, v, dk, dv [total_k, Hkv, d] bf16;
+ *   lse [Hq, total_q] f32.
+ *   cu_seqlens_q, cu_seqlens_k: DEVICE int32 arrays of B + 1 offsets,
+ *   non-decreasing, starting at 0 and ending at total_q / total_k. Sequence b
+ *   is rows cu_seqlens_q[b] .. cu_seqlens_q[b+1] of q and cu_seqlens_k[b] ..
+ *   cu_seqlens_k[b+1] of k and v, and attends only within itself, with its
+ *   own Nq_b and Nk_b: causal, window and softcap as in attn_fwd_masked, per
+ *   sequence (bottom-right alignment with off_b = Nk_b - Nq_b).
+ *   max_seqlen_q/k: the longest sequence (sizes the grid). Every Nq_b must be
+ *   <= max_seqlen_q and every Nk_b <= max_seqlen_k.
+ *   Backward workspace: attn_bwd_workspace_size(B, Hq, max_seqlen_q, d) bytes.
+ * The offsets are read on the GPU, so the host cannot check them. Offsets
+ * that break the rules above are clipped into range (no access leaves the
+ * tensors) and the next attn_check_status() returns ATTN_ERR_ARG; results
+ * of the affected sequences are then undefined. Rows that belong to no
+ * sequence (past cu_seqlens_q[B]) are not written. Sequences with Nk_b = 0
+ * get o = 0, lse = -inf and dq = 0; keys no query sees get dk = dv = 0.
+ * Errors otherwise as in attn_fwd / attn_bwd.
+ */
+attn_status attn_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* lse,
+                            const int* cu_seqlens_q, const int* cu_seqlens_k, int B, int Hq,
+                            int Hkv, int total_q, int total_k, int max_seqlen_q,
+                            int max_seqlen_k, int d, float scale, int causal, int window_left,
+                            int window_right, float softcap, attn_stream_t stream);
+
+attn_status attn_bwd_varlen(const void* q, const void* k, const void* v, const void* o,
+                            const float* lse, const void* dO, void* dq, void* dk, void* dv,
+                            const int* cu_seqlens_q, const int* cu_seqlens_k, void* workspace,
+                            size_t workspace_bytes, int B, int Hq, int Hkv, int total_q,
+                            int total_k, int max_seqlen_q, int max_seqlen_k, int d, float scale,
+                            int causal, int window_left, int window_right, float softcap,
+                            attn_stream_t stream);
 
 /*
  * Synchronises `stream`, then reads and clears the device status word.
  * Returns ATTN_ERR_TIMEOUT if a kernel gave up on a wait since the last
- * check, ATTN_ERR_CUDA on a CUDA error, and ATTN_OK otherwise.
+ * check, ATTN_ERR_ARG if a varlen call met invalid cu_seqlens offsets,
+ * ATTN_ERR_CUDA on a CUDA error, and ATTN_OK otherwise.
  */
 attn_status attn_check_status(attn_stream_t stream);
 
@@ -206,7 +250,7 @@ void attn_profile_enable(int on);
 void attn_profile_reset(void);
 attn_status attn_profile_read(int kernel, const char** name, int* launches, double* total_ms);
 
-/* ABI version of this header: major * 100 + minor (1.01: the masked calls). */
+/* ABI version of this header: major * 100 + minor (1.02: masked, softcap and varlen calls). */
 int attn_abi_version(void);
 
 #ifdef __cplusplus

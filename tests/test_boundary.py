@@ -37,7 +37,7 @@ def test_library_exports_every_declared_symbol(lib):
     for name in declared_functions():
         assert hasattr(lib, name), name
     assert set(declared_functions()) <= set(ea.SIGNATURES)
-    assert lib.attn_abi_version() == 101
+    assert lib.attn_abi_version() == 102
 
 
 FAKE = 1 << 20          # aligned, non-null, but not device memory
@@ -120,17 +120,18 @@ def test_binding_rejects_cpu_tensors():
 
 
 def fwd_masked(lib, q=FAKE, k=FAKE, v=FAKE, o=FAKE, lse=FAKE, B=1, Hq=2, Hkv=1, Nq=128, Nk=256,
-               d=64, scale=0.125, causal=0, wl=-1, wr=-1):
-    return lib.attn_fwd_masked(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, scale, causal, wl, wr, None)
+               d=64, scale=0.125, causal=0, wl=-1, wr=-1, softcap=0.0):
+    return lib.attn_fwd_masked(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, scale, causal, wl, wr,
+                               softcap, None)
 
 
 def bwd_masked(lib, ws=FAKE, ws_bytes=1 << 30, B=1, Hq=2, Hkv=1, Nq=128, Nk=256, d=64,
-               scale=0.125, causal=0, wl=-1, wr=-1, **ptrs):
+               scale=0.125, causal=0, wl=-1, wr=-1, softcap=0.0, **ptrs):
     p = {n: FAKE for n in ("q", "k", "v", "o", "lse", "dO", "dq", "dk", "dv")}
     p.update(ptrs)
     return lib.attn_bwd_masked(p["q"], p["k"], p["v"], p["o"], p["lse"], p["dO"], p["dq"],
                                p["dk"], p["dv"], ws, ws_bytes, B, Hq, Hkv, Nq, Nk, d, scale,
-                               causal, wl, wr, None)
+                               causal, wl, wr, softcap, None)
 
 
 @pytest.mark.parametrize("kw,code", [
@@ -143,6 +144,9 @@ def bwd_masked(lib, ws=FAKE, ws_bytes=1 << 30, B=1, Hq=2, Hkv=1, Nq=128, Nk=256,
     (dict(q=None), ea.ATTN_ERR_ARG),
     (dict(v=FAKE + 2), ea.ATTN_ERR_ARG),
     (dict(o=None, Nk=0), ea.ATTN_ERR_ARG),        # Nk == 0 still writes o and lse
+    (dict(softcap=-1.0), ea.ATTN_ERR_ARG),
+    (dict(softcap=float("inf")), ea.ATTN_ERR_ARG),
+    (dict(softcap=float("nan")), ea.ATTN_ERR_ARG),
 ])
 def test_fwd_masked_argument_errors(lib, kw, code):
     assert fwd_masked(lib, **kw) == code
@@ -187,3 +191,72 @@ def test_bwd_masked_workspace_is_sized_by_queries(lib):
     need = lib.attn_bwd_workspace_size(1, 2, 128, 64)
     # Exactly the Nq-sized workspace passes the argument checks (then: no device).
     assert bwd_masked(lib, Nq=128, Nk=4096, ws_bytes=need) == ea.ATTN_ERR_CUDA
+
+
+CU = 1 << 21            # 4-byte aligned, non-null, but not device memory
+
+
+def fwd_varlen(lib, q=FAKE, k=FAKE, v=FAKE, o=FAKE, lse=FAKE, cu_q=CU, cu_k=CU, B=2, Hq=2, Hkv=1,
+               total_q=300, total_k=500, max_q=200, max_k=300, d=128, scale=0.1, causal=1,
+               wl=-1, wr=-1, softcap=0.0):
+    return lib.attn_fwd_varlen(q, k, v, o, lse, cu_q, cu_k, B, Hq, Hkv, total_q, total_k, max_q,
+                               max_k, d, scale, causal, wl, wr, softcap, None)
+
+
+def bwd_varlen(lib, ws=FAKE, ws_bytes=1 << 30, cu_q=CU, cu_k=CU, B=2, Hq=2, Hkv=1, total_q=300,
+               total_k=500, max_q=200, max_k=300, d=128, scale=0.1, causal=1, wl=-1, wr=-1,
+               softcap=0.0, **ptrs):
+    p = {n: FAKE for n in ("q", "k", "v", "o", "lse", "dO", "dq", "dk", "dv")}
+    p.update(ptrs)
+    return lib.attn_bwd_varlen(p["q"], p["k"], p["v"], p["o"], p["lse"], p["dO"], p["dq"],
+                               p["dk"], p["dv"], cu_q, cu_k, ws, ws_bytes, B, Hq, Hkv, total_q,
+                               total_k, max_q, max_k, d, scale, causal, wl, wr, softcap, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(total_q=-1), ea.ATTN_ERR_ARG),
+    (dict(total_k=-5), ea.ATTN_ERR_ARG),
+    (dict(max_q=0), ea.ATTN_ERR_ARG),                # rows but no room for them
+    (dict(max_k=-1), ea.ATTN_ERR_ARG),
+    (dict(max_q=(1 << 24) + 1), ea.ATTN_ERR_ARG),
+    (dict(B=-1), ea.ATTN_ERR_ARG),
+    (dict(Hq=3, Hkv=2), ea.ATTN_ERR_ARG),
+    (dict(d=96), ea.ATTN_ERR_UNSUPPORTED),
+    (dict(softcap=-2.0), ea.ATTN_ERR_ARG),
+    (dict(causal=5), ea.ATTN_ERR_ARG),
+    (dict(q=None), ea.ATTN_ERR_ARG),
+    (dict(lse=FAKE + 4), ea.ATTN_ERR_ARG),
+])
+def test_fwd_varlen_argument_errors(lib, kw, code):
+    assert fwd_varlen(lib, **kw) == code
+    assert lib.attn_get_last_error().decode() != ""
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(total_q=-1), ea.ATTN_ERR_ARG),
+    (dict(ws=None), ea.ATTN_ERR_ARG),
+    (dict(ws_bytes=2 * 2 * 256 * 4 - 4), ea.ATTN_ERR_ARG),   # sized by B, Hq and max_seqlen_q
+    (dict(dk=None), ea.ATTN_ERR_ARG),
+    (dict(softcap=float("nan")), ea.ATTN_ERR_ARG),
+])
+def test_bwd_varlen_argument_errors(lib, kw, code):
+    assert bwd_varlen(lib, **kw) == code
+
+
+def test_varlen_empty_batches(lib):
+    assert fwd_varlen(lib, B=0, q=None, k=None, v=None, o=None, lse=None, cu_q=None,
+                      cu_k=None) == ea.ATTN_OK
+    assert fwd_varlen(lib, total_q=0, q=None, o=None, lse=None) == ea.ATTN_OK
+    assert bwd_varlen(lib, total_q=0, total_k=0) == ea.ATTN_OK
+
+
+def test_varlen_offsets_checks(lib):
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    # Valid arguments: without a device the call fails as a CUDA error. Null or
+    # misaligned offsets are argument errors found on the host.
+    assert fwd_varlen(lib) == ea.ATTN_ERR_CUDA
+    assert fwd_varlen(lib, cu_q=None) == ea.ATTN_ERR_ARG
+    assert fwd_varlen(lib, cu_k=CU + 2) == ea.ATTN_ERR_ARG
+    assert bwd_varlen(lib, cu_k=None) == ea.ATTN_ERR_ARG

@@ -113,3 +113,28 @@ def make_inputs_qk(B: int, Hq: int, Hkv: int, Nq: int, Nk: int, d: int, seed: in
     if with_grad_out:
         out.append(torch.randn((B, Hq, Nq, d), generator=g, dtype=torch.float32).to(torch.bfloat16))
     return tuple(out)
+
+
+def make_packed_inputs(lens_q, lens_k, Hq: int, Hkv: int, d: int, seed: int,
+                       q_mult: float = 1.0, with_grad_out: bool = True):
+    """A packed (varlen) batch: (q, k, v[, dO], cu_q, cu_k) on the CPU.
+
+    q/dO are [sum(lens_q), Hq, d] and k/v [sum(lens_k), Hkv, d], bfloat16,
+    drawn like ``make_inputs`` (one generator seeded with ``seed``, order
+    Q, K, V, dO, float32 normal rounded once). cu_q/cu_k are int32 offsets of
+    length B + 1 starting at 0.
+    """
+    if len(lens_q) != len(lens_k):
+        raise ValueError("lens_q and lens_k must have the same length")
+    tq, tk = int(sum(lens_q)), int(sum(lens_k))
+    g = torch.Generator(device="cpu").manual_seed(seed)
+    q = torch.randn((tq, Hq, d), generator=g, dtype=torch.float32)
+    k = torch.randn((tk, Hkv, d), generator=g, dtype=torch.float32)
+    v = torch.randn((tk, Hkv, d), generator=g, dtype=torch.float32)
+    out = [(q * q_mult).to(torch.bfloat16), k.to(torch.bfloat16), v.to(torch.bfloat16)]
+    if with_grad_out:
+        out.append(torch.randn((tq, Hq, d), generator=g, dtype=torch.float32).to(torch.bfloat16))
+    cu = lambda lens: torch.tensor([0] + list(torch.cumsum(torch.tensor(lens), 0).tolist()),
+                                   dtype=torch.int32)
+    out += [cu(lens_q), cu(lens_k)]
+    return tuple(out)
