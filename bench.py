@@ -280,6 +280,81 @@ def run_reference(args):
 
 # ------------------------------------------------------------------ ours
 
+def visible_pairs(n_q, n_k, causal, window=(-1, -1)):
+    """Number of (query, key) pairs the mask keeps for one head: bottom-right
+    alignment, off = Nk - Nq; window (left, right), negative = unbounded."""
+    import numpy as np
+    i = np.arange(n_q, dtype=np.int64)
+    off = n_k - n_q
+    lo = i + off - window[0] if window[0] >= 0 else np.zeros_like(i)
+    hi = np.full_like(i, n_k - 1)
+    if causal:
+        hi = np.minimum(hi, i + off)
+    if window[1] >= 0:
+        hi = np.minimum(hi, i + off + window[1])
+    return int(np.maximum(0, np.minimum(n_k - 1, hi) - np.maximum(0, lo) + 1).sum())
+
+
+def variant_targets(ea, torch, peak, iters=5, warmup=2):
+    """Forward + backward TFLOP/s (14 d FLOPs per visible pair) of the variant
+    paths: sliding window, Nq != Nk, softcapping and a packed varlen batch."""
+    import numpy as np
+    out = []
+
+    def timed(name, step, pairs, d):
+        for _ in range(warmup):
+            step()
+        ea.attn_check_status()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        a.record()
+        for _ in range(iters):
+            step()
+        b.record()
+        torch.cuda.synchronize()
+        ea.attn_check_status()
+        ms = a.elapsed_time(b) / iters
+        tf = 14.0 * d * pairs / ms / 1e9
+        out.append({"workload": name, "ms": ms, "tflops": tf, "frac_of_measured_peak": tf / peak})
+
+    fixed = [("swa1024_causal_B4_H16_N4096_d128", 4, 16, 4096, 4096, True, (1024, 0), 0.0),
+             ("chunk_causal_B4_H16_Nq2048_Nk8192_d128", 4, 16, 2048, 8192, True, (-1, -1), 0.0),
+             ("softcap50_causal_B4_H16_N4096_d128", 4, 16, 4096, 4096, True, (-1, -1), 50.0)]
+    for name, B, H, Nq, Nk, causal, win, cap in fixed:
+        q, k, v, do = (t.cuda() for t in workloads.make_inputs_qk(B, H, H, Nq, Nk, 128, seed=7))
+        o, lse = torch.empty_like(q), torch.empty((B, H, Nq), dtype=torch.float32, device="cuda")
+        dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+        ws = torch.empty(ea.attn_bwd_workspace_size(B, H, Nq, 128), dtype=torch.uint8,
+                         device="cuda")
+
+        def step():
+            ea.attn_fwd_masked(q, k, v, o, lse, causal=causal, window=win, softcap=cap)
+            ea.attn_bwd_masked(q, k, v, o, lse, do, dq, dk, dv, ws, causal=causal, window=win,
+                               softcap=cap)
+        timed(name, step, B * H * visible_pairs(Nq, Nk, causal, win), 128)
+        del q, k, v, do, o, lse, dq, dk, dv, ws
+        torch.cuda.empty_cache()
+
+    lens = [int(x) for x in np.random.default_rng(0).integers(256, 4097, 16)]
+    H = 16
+    q, k, v, do, cq, ck = (t.cuda() for t in workloads.make_packed_inputs(lens, lens, H, H, 128,
+                                                                          seed=8))
+    o, lse = torch.empty_like(q), torch.empty((H, q.shape[0]), dtype=torch.float32, device="cuda")
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    mx = max(lens)
+    ws = torch.empty(ea.attn_bwd_workspace_size(len(lens), H, mx, 128), dtype=torch.uint8,
+                     device="cuda")
+
+    def vstep():
+        ea.attn_fwd_varlen(q, k, v, cq, ck, mx, mx, o, lse, causal=True)
+        ea.attn_bwd_varlen(q, k, v, o, lse, do, cq, ck, mx, mx, dq, dk, dv, ws, causal=True)
+    timed(f"varlen16_causal_H16_d128_total{sum(lens)}", vstep,
+          H * sum(visible_pairs(n, n, True) for n in lens), 128)
+    del q, k, v, do, o, lse, dq, dk, dv, ws
+    torch.cuda.empty_cache()
+    return out
+
+
 def fwd_target(ea, torch, w, iters=10, warmup=3):
     """Forward-only TFLOP/s on one workload (inputs resident, > L2)."""
     q, k, v = (t.cuda() for t in workloads.make_inputs(w, with_grad_out=False))
@@ -424,6 +499,7 @@ def run_ours(args):
            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps}
 
     extra = None
+    variants = None
     if not args.no_extra and rank == 0 and not fwd_only:
         del pin, outs
         torch.cuda.empty_cache()
@@ -432,6 +508,7 @@ def run_ours(args):
             r = fwd_target(ea, torch, tw)
             r["frac_of_measured_peak"] = r["tflops"] / peaks["bf16_tflops"]
             extra.append(r)
+        variants = variant_targets(ea, torch, peaks["bf16_tflops"])
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline and not fwd_only:
@@ -452,6 +529,7 @@ def run_ours(args):
             "frac_of_peak": value / peaks["bf16_tflops"],
             "roofline": roofline, "kernels": kernels, "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": launches, "clocks": clocks, "fwd_targets": extra,
+            "variants_fwd_bwd": variants,
             "kernel_source_sha": kernel_source_sha()}
     print(json.dumps(line), flush=True)
     return 0
