@@ -212,7 +212,19 @@ def oracle_baseline(w, inputs, steps, per_step_s, warmup=1):
     return {"value": flops / dt / 1e12, "unit": UNIT, "cores": cpu_threads(), "kind": "oracle",
             "sample": f"float64 numpy oracle, fwd+bwd of the last {rows} query rows of one head "
                       f"(all {w.N} keys, causal) per step, {steps} steps over rotating heads",
-            "seconds": dt, "rows_per_step": rows}
+            "seconds": dt, "rows_per_step": rows, "gflops": flops / dt / 1e9,
+            "blas": blas_info()}
+
+
+def blas_info():
+    """The BLAS library numpy uses and its thread count, as threadpoolctl reports it."""
+    try:
+        from threadpoolctl import threadpool_info
+        libs = [f"{d.get('internal_api')} {d.get('version')} ({d.get('num_threads')} threads)"
+                for d in threadpool_info() if d.get("user_api") == "blas"]
+        return "; ".join(libs) or None
+    except Exception:   # informational only
+        return None
 
 
 # ------------------------------------------------------------------ distributed
@@ -355,6 +367,59 @@ def variant_targets(ea, torch, peak, iters=5, warmup=2):
     return out
 
 
+def small_target(ea, torch, w, hbm_gbs, iters=50, warmup=5):
+    """The small configurations are latency-bound. Reports microseconds per
+    forward and per forward + backward, called through the API from Python
+    (host overhead included) and replayed from a CUDA graph that captured the
+    same calls (device time only), plus the forward's HBM byte rate (q, k, v
+    read and o, lse written once) from the graph timing."""
+    q, k, v, do = (t.cuda() for t in workloads.make_inputs(w, with_grad_out=True))
+    o = torch.empty_like(q)
+    lse = torch.empty(q.shape[:3], dtype=torch.float32, device="cuda")
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    ws = torch.empty(max(16, ea.attn_bwd_workspace_size(w.B, w.Hq, w.N, w.d)), dtype=torch.uint8,
+                     device="cuda")
+
+    def fwd():
+        ea.attn_fwd(q, k, v, o, lse, scale=w.scale, causal=w.causal)
+
+    def fwd_bwd():
+        fwd()
+        ea.attn_bwd(q, k, v, o, lse, do, dq, dk, dv, ws, scale=w.scale, causal=w.causal)
+
+    def timed(fn):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        a.record()
+        for _ in range(iters):
+            fn()
+        b.record()
+        torch.cuda.synchronize()
+        ea.attn_check_status()
+        return a.elapsed_time(b) / iters * 1e3
+
+    res = {"workload": w.name}
+    for name, fn in (("fwd", fwd), ("fwd_bwd", fwd_bwd)):
+        for _ in range(warmup):
+            fn()
+        res[f"{name}_api_us"] = timed(fn)
+        g = torch.cuda.CUDAGraph()
+        side = torch.cuda.Stream()
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):
+            fn()
+        torch.cuda.current_stream().wait_stream(side)
+        with torch.cuda.graph(g, capture_error_mode="relaxed"):
+            fn()
+        res[f"{name}_graph_us"] = timed(g.replay)
+        del g
+    fwd_bytes = 2.0 * w.d * (2 * w.B * w.Hq * w.N + 2 * w.B * w.Hkv * w.N) + 4.0 * w.B * w.Hq * w.N
+    res["fwd_hbm_gbs"] = fwd_bytes / (res["fwd_graph_us"] * 1e-6) / 1e9
+    res["fwd_hbm_frac_of_measured"] = res["fwd_hbm_gbs"] / hbm_gbs
+    res["fwd_bwd_tflops"] = (w.fwd_flops() + w.bwd_flops()) / (res["fwd_bwd_graph_us"] * 1e-6) / 1e12
+    return res
+
+
 def fwd_target(ea, torch, w, iters=10, warmup=3):
     """Forward-only TFLOP/s on one workload (inputs resident, > L2)."""
     q, k, v = (t.cuda() for t in workloads.make_inputs(w, with_grad_out=False))
@@ -417,11 +482,12 @@ def run_ours(args):
     ea.profile_reset()
     ea.profile_enable(True)
     sampler.start()
-    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
+    ev0, ev1 = evs[0], evs[-1]
     ev0.record(stream)
-    for _ in range(args.steps):
+    for n_step in range(args.steps):
         step()
-    ev1.record(stream)
+        evs[n_step + 1].record(stream)
     torch.cuda.synchronize()
     sampler.stop()
     ea.profile_enable(False)
@@ -429,8 +495,19 @@ def run_ours(args):
         dist.barrier()
     ea.attn_check_status()
     elapsed = max_over_ranks(ev0.elapsed_time(ev1), dist, "cuda")
+    per_step = sorted(evs[n].elapsed_time(evs[n + 1]) for n in range(args.steps))
+    pick = lambda f: per_step[min(len(per_step) - 1, int(f * len(per_step)))]  # noqa: E731
+    step_dist = {"p10_ms": pick(0.10), "median_ms": pick(0.50), "p90_ms": pick(0.90),
+                 "rank": rank}
     prof = ea.profile_read()
     launches = sum(n for n, _ in prof.values())
+    # Forward and backward separately, from the same timed region.
+    fwd_ms = prof["fwd_kernel"][1] / max(1, prof["fwd_kernel"][0])
+    bwd_ms = sum(prof[k2][1] for k2 in ("bwd_pre_kernel", "bwd_dkdv_kernel", "bwd_dq_kernel")) \
+        / max(1, prof["bwd_dkdv_kernel"][0])
+    split = {"fwd_ms": fwd_ms, "fwd_tflops": w.fwd_flops() / fwd_ms / 1e9}
+    if not fwd_only:
+        split.update({"bwd_ms": bwd_ms, "bwd_tflops": w.bwd_flops() / bwd_ms / 1e9})
 
     flops_step = w.fwd_flops() + (0.0 if fwd_only else w.bwd_flops())
     value = job_throughput(flops_step, args.steps, world, elapsed)
@@ -536,6 +613,7 @@ def run_ours(args):
 
     extra = None
     variants = None
+    small = None
     if not args.no_extra and rank == 0 and not fwd_only:
         del pin, host_out
         torch.cuda.empty_cache()
@@ -545,6 +623,7 @@ def run_ours(args):
             r["frac_of_measured_peak"] = r["tflops"] / peaks["bf16_tflops"]
             extra.append(r)
         variants = variant_targets(ea, torch, peaks["bf16_tflops"])
+        small = [small_target(ea, torch, tw, peaks["hbm_gbs"]) for tw in (workloads.C1, workloads.C2)]
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline and not fwd_only:
@@ -563,9 +642,11 @@ def run_ours(args):
             "data": "synthetic (seeded iid N(0,1) -> bf16)",
             "config": dict(config_dict(w, world), mode=args.mode),
             "frac_of_peak": value / peaks["bf16_tflops"],
+            "frac_of_nominal_2250": value / 2250.0,
+            "step_distribution": step_dist, "fwd_bwd_split": split,
             "roofline": roofline, "kernels": kernels, "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": launches, "clocks": clocks, "fwd_targets": extra,
-            "variants_fwd_bwd": variants,
+            "variants_fwd_bwd": variants, "small_configs": small,
             "kernel_source_sha": kernel_source_sha()}
     print(json.dumps(line), flush=True)
     return 0
