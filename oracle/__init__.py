@@ -5,6 +5,7 @@ leg may import this package; the CUDA library never does.
 """
 from .attention_ref import (  # noqa: F401
     attention_backward,
+    attention_backward_dq_rows,
     attention_backward_varlen,
     attention_bruteforce,
     attention_forward,

@@ -275,6 +275,33 @@ def attention_backward(q, k, v, do, scale: float, causal: bool, heads=None, wind
     return dq, dk, dv
 
 
+def attention_backward_dq_rows(q, k, v, do, scale: float, causal: bool, b: int, hq: int, rows,
+                               window=(-1, -1), softcap: float = 0.0):
+    """dQ of the listed query rows of head (b, hq), for full-size spot checks.
+
+    Every quantity dQ needs is local to the row: its scores over all keys,
+    P from their softmax, dP = dO_row V^T, D = sum(P * dP), dS = P * (dP - D)
+    (times 1 - tanh^2 with softcapping) and dQ = scale * dS K.
+    """
+    Hq, Nq = q.shape[1], q.shape[2]
+    hk = _kv_head(hq, Hq, k.shape[1])
+    rows = np.asarray(rows)
+    qr = to_f64(q[b, hq][rows])
+    kk, vv = to_f64(k[b, hk]), to_f64(v[b, hk])
+    dor = to_f64(do[b, hq][rows])
+    z = (qr @ kk.T) * scale
+    s = capped(z, softcap)
+    if causal or window[0] >= 0 or window[1] >= 0:
+        s = np.where(visible(rows, Nq, kk.shape[0], causal, window), s, -np.inf)
+    p, _, _ = softmax_rows(s)
+    dp = dor @ vv.T
+    ds = p * (dp - np.sum(p * dp, axis=1, keepdims=True))
+    if softcap > 0:
+        t = np.tanh(z / softcap)
+        ds = ds * (1.0 - t * t)
+    return scale * (ds @ kk)
+
+
 # --------------------------------------------------------------------------
 # The tiled algorithm, restated separately so tests can pin it to the
 # definition. unite.ai "Was ist FlashAttention?", section "Eine fuenfstufige

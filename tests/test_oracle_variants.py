@@ -269,3 +269,30 @@ def test_varlen_rejects_bad_offsets(cu):
     q = rand(3, 1, 2)
     with pytest.raises(ValueError):
         oracle.attention_forward_varlen(q, q, q, cu, [0, 3] if len(cu) == 2 else [0, 1, 3], 1.0, False)
+
+
+# ---------------------------------------------------------------- row-wise dQ
+
+@pytest.mark.parametrize("causal,window,softcap", [(True, (-1, -1), 0.0), (False, (3, 2), 0.0),
+                                                   (True, (-1, -1), 1.5)])
+def test_dq_rows_equal_the_full_backward(causal, window, softcap):
+    """The row-wise dQ used for full-size spot checks is the same gradient the
+    whole-head backward gives (which central differences pin above)."""
+    B, Hq, Hkv, N, d = 1, 4, 2, 23, 8
+    q, k, v, do = rand(B, Hq, N, d), rand(B, Hkv, N, d), rand(B, Hkv, N, d), rand(B, Hq, N, d)
+    dq, _, _ = oracle.attention_backward(q, k, v, do, 0.6, causal, window=window, softcap=softcap)
+    rows = [0, 1, 7, 21, 22]
+    for b, h in ((0, 0), (0, 3)):
+        got = oracle.attention_backward_dq_rows(q, k, v, do, 0.6, causal, b, h, rows,
+                                                window=window, softcap=softcap)
+        np.testing.assert_allclose(got, dq[b, h][rows], rtol=0, atol=1e-12)
+
+
+def test_gradient_identities_hold_in_the_oracle():
+    """Identities the GPU tests use at sizes the oracle cannot run whole:
+    the weights of a row sum to one, so sum_k dV[k] = sum_q dO[q]; the entries
+    of a row of dS sum to zero, so sum_k dK[k] = 0."""
+    q, k, v, do = rand(1, 2, 30, 8), rand(1, 2, 30, 8), rand(1, 2, 30, 8), rand(1, 2, 30, 8)
+    _, dk, dv = oracle.attention_backward(q, k, v, do, 0.5, True)
+    np.testing.assert_allclose(dv.sum(axis=2), do.sum(axis=2), rtol=0, atol=1e-12)
+    np.testing.assert_allclose(dk.sum(axis=2), 0.0, rtol=0, atol=1e-12)
