@@ -89,6 +89,20 @@ def _check(status: int):
         raise AttnError(status, msg)
 
 
+def _device_guard(*tensors):
+    """All tensor arguments must live on one CUDA device. The call then runs
+    with that device current (the library launches on the current device)."""
+    import torch
+    devs = {t.device for t in tensors if isinstance(t, torch.Tensor)}
+    if len(devs) != 1:
+        raise ValueError(f"all tensors must be on one device, got {sorted(map(str, devs))}")
+    dev = devs.pop()
+    if dev.type != "cuda":
+        raise ValueError(f"tensors must be CUDA tensors (the library takes device pointers), "
+                         f"got {dev}")
+    return torch.cuda.device(dev)
+
+
 def _stream_handle(stream):
     import torch
     s = torch.cuda.current_stream() if stream is None else stream
@@ -130,9 +144,10 @@ def attn_fwd(q, k, v, o=None, lse=None, scale=None, causal=False, stream=None):
         raise ValueError("o/lse shape mismatch")
     scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
     lib = load_library()
-    _check(lib.attn_fwd(_dev_ptr(q, "q"), _dev_ptr(k, "k"), _dev_ptr(v, "v"), _dev_ptr(o, "o"),
-                        _dev_ptr(lse, "lse"), B, Hq, Hkv, N, d, scale, int(bool(causal)),
-                        _stream_handle(stream)))
+    with _device_guard(q, k, v, o, lse):
+        _check(lib.attn_fwd(_dev_ptr(q, "q"), _dev_ptr(k, "k"), _dev_ptr(v, "v"), _dev_ptr(o, "o"),
+                            _dev_ptr(lse, "lse"), B, Hq, Hkv, N, d, scale, int(bool(causal)),
+                            _stream_handle(stream)))
     return o, lse
 
 
@@ -164,11 +179,12 @@ def attn_bwd(q, k, v, o, lse, dO, dq=None, dk=None, dv=None, workspace=None, sca
         workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
     scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
     lib = load_library()
-    _check(lib.attn_bwd(_dev_ptr(q, "q"), _dev_ptr(k, "k"), _dev_ptr(v, "v"), _dev_ptr(o, "o"),
-                        _dev_ptr(lse, "lse"), _dev_ptr(dO, "dO"), _dev_ptr(dq, "dq"),
-                        _dev_ptr(dk, "dk"), _dev_ptr(dv, "dv"), _dev_ptr(workspace, "workspace"),
-                        workspace.numel() * workspace.element_size(),
-                        B, Hq, Hkv, N, d, scale, int(bool(causal)), _stream_handle(stream)))
+    with _device_guard(q, k, v, o, lse, dO, dq, dk, dv, workspace):
+        _check(lib.attn_bwd(_dev_ptr(q, "q"), _dev_ptr(k, "k"), _dev_ptr(v, "v"), _dev_ptr(o, "o"),
+                            _dev_ptr(lse, "lse"), _dev_ptr(dO, "dO"), _dev_ptr(dq, "dq"),
+                            _dev_ptr(dk, "dk"), _dev_ptr(dv, "dv"), _dev_ptr(workspace, "workspace"),
+                            workspace.numel() * workspace.element_size(),
+                            B, Hq, Hkv, N, d, scale, int(bool(causal)), _stream_handle(stream)))
     return dq, dk, dv
 
 
@@ -185,11 +201,12 @@ def attn_bwd_noalloc(q, k, v, o, lse, dO, dq, dk, dv, scale=None, causal=False, 
     Hkv = k.shape[1]
     scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
     lib = load_library()
-    _check(lib.attn_bwd_noalloc(_dev_ptr(q, "q"), _dev_ptr(k, "k"), _dev_ptr(v, "v"),
-                                _dev_ptr(o, "o"), _dev_ptr(lse, "lse"), _dev_ptr(dO, "dO"),
-                                _dev_ptr(dq, "dq"), _dev_ptr(dk, "dk"), _dev_ptr(dv, "dv"),
-                                B, Hq, Hkv, N, d, scale, int(bool(causal)),
-                                _stream_handle(stream)))
+    with _device_guard(q, k, v, o, lse, dO, dq, dk, dv):
+        _check(lib.attn_bwd_noalloc(_dev_ptr(q, "q"), _dev_ptr(k, "k"), _dev_ptr(v, "v"),
+                                    _dev_ptr(o, "o"), _dev_ptr(lse, "lse"), _dev_ptr(dO, "dO"),
+                                    _dev_ptr(dq, "dq"), _dev_ptr(dk, "dk"), _dev_ptr(dv, "dv"),
+                                    B, Hq, Hkv, N, d, scale, int(bool(causal)),
+                                    _stream_handle(stream)))
     return dq, dk, dv
 
 
@@ -228,10 +245,11 @@ def attn_fwd_masked(q, k, v, o=None, lse=None, scale=None, causal=False, window=
     scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
     wl, wr = _window(window)
     lib = load_library()
-    _check(lib.attn_fwd_masked(_dev_ptr(q, "q"), _dev_ptr(k, "k"), _dev_ptr(v, "v"),
-                               _dev_ptr(o, "o"), _dev_ptr(lse, "lse"), B, Hq, Hkv, Nq, Nk, d,
-                               scale, int(bool(causal)), wl, wr, _softcap(softcap),
-                               _stream_handle(stream)))
+    with _device_guard(q, k, v, o, lse):
+        _check(lib.attn_fwd_masked(_dev_ptr(q, "q"), _dev_ptr(k, "k"), _dev_ptr(v, "v"),
+                                   _dev_ptr(o, "o"), _dev_ptr(lse, "lse"), B, Hq, Hkv, Nq, Nk, d,
+                                   scale, int(bool(causal)), wl, wr, _softcap(softcap),
+                                   _stream_handle(stream)))
     return o, lse
 
 
@@ -260,13 +278,14 @@ def attn_bwd_masked(q, k, v, o, lse, dO, dq=None, dk=None, dv=None, workspace=No
     scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
     wl, wr = _window(window)
     lib = load_library()
-    _check(lib.attn_bwd_masked(_dev_ptr(q, "q"), _dev_ptr(k, "k"), _dev_ptr(v, "v"),
-                               _dev_ptr(o, "o"), _dev_ptr(lse, "lse"), _dev_ptr(dO, "dO"),
-                               _dev_ptr(dq, "dq"), _dev_ptr(dk, "dk"), _dev_ptr(dv, "dv"),
-                               _dev_ptr(workspace, "workspace"),
-                               workspace.numel() * workspace.element_size(),
-                               B, Hq, Hkv, Nq, Nk, d, scale, int(bool(causal)), wl, wr,
-                               _softcap(softcap), _stream_handle(stream)))
+    with _device_guard(q, k, v, o, lse, dO, dq, dk, dv, workspace):
+        _check(lib.attn_bwd_masked(_dev_ptr(q, "q"), _dev_ptr(k, "k"), _dev_ptr(v, "v"),
+                                   _dev_ptr(o, "o"), _dev_ptr(lse, "lse"), _dev_ptr(dO, "dO"),
+                                   _dev_ptr(dq, "dq"), _dev_ptr(dk, "dk"), _dev_ptr(dv, "dv"),
+                                   _dev_ptr(workspace, "workspace"),
+                                   workspace.numel() * workspace.element_size(),
+                                   B, Hq, Hkv, Nq, Nk, d, scale, int(bool(causal)), wl, wr,
+                                   _softcap(softcap), _stream_handle(stream)))
     return dq, dk, dv
 
 
@@ -306,11 +325,12 @@ def attn_fwd_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, max_seqle
     scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
     wl, wr = _window(window)
     lib = load_library()
-    _check(lib.attn_fwd_varlen(_dev_ptr(q, "q"), _dev_ptr(k, "k"), _dev_ptr(v, "v"),
-                               _dev_ptr(o, "o"), _dev_ptr(lse, "lse"), cq, ck, B, Hq, Hkv,
-                               total_q, total_k, int(max_seqlen_q), int(max_seqlen_k), d, scale,
-                               int(bool(causal)), wl, wr, _softcap(softcap),
-                               _stream_handle(stream)))
+    with _device_guard(q, k, v, o, lse, cu_seqlens_q, cu_seqlens_k):
+        _check(lib.attn_fwd_varlen(_dev_ptr(q, "q"), _dev_ptr(k, "k"), _dev_ptr(v, "v"),
+                                   _dev_ptr(o, "o"), _dev_ptr(lse, "lse"), cq, ck, B, Hq, Hkv,
+                                   total_q, total_k, int(max_seqlen_q), int(max_seqlen_k), d, scale,
+                                   int(bool(causal)), wl, wr, _softcap(softcap),
+                                   _stream_handle(stream)))
     return o, lse
 
 
@@ -345,14 +365,15 @@ def attn_bwd_varlen(q, k, v, o, lse, dO, cu_seqlens_q, cu_seqlens_k, max_seqlen_
     scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
     wl, wr = _window(window)
     lib = load_library()
-    _check(lib.attn_bwd_varlen(_dev_ptr(q, "q"), _dev_ptr(k, "k"), _dev_ptr(v, "v"),
-                               _dev_ptr(o, "o"), _dev_ptr(lse, "lse"), _dev_ptr(dO, "dO"),
-                               _dev_ptr(dq, "dq"), _dev_ptr(dk, "dk"), _dev_ptr(dv, "dv"), cq, ck,
-                               _dev_ptr(workspace, "workspace"),
-                               workspace.numel() * workspace.element_size(), B, Hq, Hkv, total_q,
-                               total_k, int(max_seqlen_q), int(max_seqlen_k), d, scale,
-                               int(bool(causal)), wl, wr, _softcap(softcap),
-                               _stream_handle(stream)))
+    with _device_guard(q, k, v, o, lse, dO, dq, dk, dv, workspace, cu_seqlens_q, cu_seqlens_k):
+        _check(lib.attn_bwd_varlen(_dev_ptr(q, "q"), _dev_ptr(k, "k"), _dev_ptr(v, "v"),
+                                   _dev_ptr(o, "o"), _dev_ptr(lse, "lse"), _dev_ptr(dO, "dO"),
+                                   _dev_ptr(dq, "dq"), _dev_ptr(dk, "dk"), _dev_ptr(dv, "dv"), cq, ck,
+                                   _dev_ptr(workspace, "workspace"),
+                                   workspace.numel() * workspace.element_size(), B, Hq, Hkv, total_q,
+                                   total_k, int(max_seqlen_q), int(max_seqlen_k), d, scale,
+                                   int(bool(causal)), wl, wr, _softcap(softcap),
+                                   _stream_handle(stream)))
     return dq, dk, dv
 
 

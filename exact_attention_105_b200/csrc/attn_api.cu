@@ -97,44 +97,89 @@ using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t
                                    CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
 EncodeTiledFn g_encode = nullptr;
-int g_num_sms = 148;
 attn_status g_init_status = ATTN_OK;
 char g_init_msg[256] = "";
 std::once_flag g_init_once;
 
+// Devices a process may use (per-device caches below are indexed by ordinal).
+constexpr int kMaxDevices = 64;
+
 void init_once() {
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) {
-    g_init_status = ATTN_ERR_CUDA;
-    snprintf(g_init_msg, sizeof(g_init_msg), "no CUDA device: %s", cudaGetErrorString(e));
-    return;
-  }
-  cudaDeviceProp prop;
-  e = cudaGetDeviceProperties(&prop, dev);
-  if (e != cudaSuccess || prop.major != 10 || prop.minor != 0) {
-    g_init_status = ATTN_ERR_CUDA;
-    snprintf(g_init_msg, sizeof(g_init_msg),
-             "this library is built for sm_100a (B200); device %d is sm_%d%d", dev, prop.major,
-             prop.minor);
-    return;
-  }
   cudaDriverEntryPointQueryResult q;
   void* fn = nullptr;
-  e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q);
+  cudaError_t e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q);
   if (e != cudaSuccess || q != cudaDriverEntryPointSuccess || fn == nullptr) {
     g_init_status = ATTN_ERR_CUDA;
-    snprintf(g_init_msg, sizeof(g_init_msg), "cuTensorMapEncodeTiled unavailable");
+    snprintf(g_init_msg, sizeof(g_init_msg), "cuTensorMapEncodeTiled unavailable (%s)",
+             cudaGetErrorString(e));
     return;
   }
   g_encode = reinterpret_cast<EncodeTiledFn>(fn);
-  g_num_sms = prop.multiProcessorCount > 0 ? prop.multiProcessorCount : 148;
+}
+
+// The current device must be an sm_100 part; checked once per device.
+attn_status check_device() {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return fail(ATTN_ERR_CUDA, "no CUDA device: %s", cudaGetErrorString(e));
+  }
+  if (dev < 0 || dev >= kMaxDevices) return fail(ATTN_ERR_CUDA, "device index %d unsupported", dev);
+  static std::mutex mu;
+  static int arch[kMaxDevices] = {};          // 0: not checked yet, else major * 10 + minor
+  std::lock_guard<std::mutex> g(mu);
+  if (arch[dev] == 0) {
+    cudaDeviceProp prop;
+    e = cudaGetDeviceProperties(&prop, dev);
+    if (e != cudaSuccess) {
+      cudaGetLastError();
+      return fail(ATTN_ERR_CUDA, "cudaGetDeviceProperties(%d): %s", dev, cudaGetErrorString(e));
+    }
+    arch[dev] = prop.major * 10 + prop.minor;
+  }
+  if (arch[dev] != 100)
+    return fail(ATTN_ERR_CUDA, "this library is built for sm_100a (B200); device %d is sm_%d", dev,
+                arch[dev]);
+  return ATTN_OK;
 }
 
 attn_status ensure_init() {
+  attn_status st = check_device();
+  if (st != ATTN_OK) return st;
   std::call_once(g_init_once, init_once);
   if (g_init_status != ATTN_OK) return fail(g_init_status, "%s", g_init_msg);
   return ATTN_OK;
+}
+
+// One-time setup of a kernel on each device it runs on: the dynamic shared
+// memory opt-in applies to the device current when it is made. Also records
+// the register count ptxas gave the kernel (the forward checks it against its
+// setmaxnreg split).
+struct KernelSetup {
+  std::mutex mu;
+  bool done[kMaxDevices] = {};
+  cudaError_t err[kMaxDevices] = {};
+  int regs[kMaxDevices] = {};
+};
+
+template <typename Kern>
+cudaError_t prepare_kernel(Kern kern, int smem_bytes, KernelSetup& ks, int* regs = nullptr) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> g(ks.mu);
+  if (!ks.done[dev]) {
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes);
+    cudaFuncAttributes fa;
+    if (e == cudaSuccess) e = cudaFuncGetAttributes(&fa, kern);
+    ks.err[dev] = e;
+    ks.regs[dev] = (e == cudaSuccess) ? fa.numRegs : 0;
+    ks.done[dev] = true;
+  }
+  if (regs) *regs = ks.regs[dev];
+  return ks.err[dev];
 }
 // 3-D tensor map (d, rows, z) over a bf16 tensor, with a box of 64 x 128 x 1
 // (one 128-row, 128-byte-wide column block) and 128-byte swizzle. Row and z
@@ -159,22 +204,35 @@ attn_status make_map(CUtensorMap* map, const void* base, int d, long long rows, 
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-// Null, alignment and memory-kind checks for the tensor arguments. A host
-// pointer handed to a kernel would fault the GPU, so it is rejected here.
+// Null, alignment, memory-kind and device checks for the tensor arguments. A
+// host pointer, or memory of another GPU than the current one, handed to a
+// kernel would fault the GPU, so both are rejected here.
+attn_status check_device_ptr(const void* ptr, const char* name) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  cudaPointerAttributes pa;
+  e = cudaPointerGetAttributes(&pa, ptr);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return fail(ATTN_ERR_ARG, "%s is not a CUDA pointer (%s)", name, cudaGetErrorName(e));
+  }
+  if (pa.type != cudaMemoryTypeDevice && pa.type != cudaMemoryTypeManaged)
+    return fail(ATTN_ERR_ARG, "%s is not device memory", name);
+  if (pa.type == cudaMemoryTypeDevice && pa.device != dev)
+    return fail(ATTN_ERR_ARG, "%s lives on device %d but the current device is %d", name,
+                pa.device, dev);
+  return ATTN_OK;
+}
+
 attn_status check_ptrs(const void* const* ptrs, const char* const* names, int n) {
   for (int i = 0; i < n; ++i) {
     if (ptrs[i] == nullptr) return fail(ATTN_ERR_ARG, "%s is null", names[i]);
     if (!aligned16(ptrs[i])) return fail(ATTN_ERR_ARG, "%s is not 16-byte aligned", names[i]);
   }
   for (int i = 0; i < n; ++i) {
-    cudaPointerAttributes pa;
-    cudaError_t e = cudaPointerGetAttributes(&pa, ptrs[i]);
-    if (e != cudaSuccess) {
-      cudaGetLastError();
-      return fail(ATTN_ERR_ARG, "%s is not a CUDA pointer (%s)", names[i], cudaGetErrorName(e));
-    }
-    if (pa.type != cudaMemoryTypeDevice && pa.type != cudaMemoryTypeManaged)
-      return fail(ATTN_ERR_ARG, "%s is not device memory", names[i]);
+    attn_status st = check_device_ptr(ptrs[i], names[i]);
+    if (st != ATTN_OK) return st;
   }
   return ATTN_OK;
 }
@@ -236,16 +294,9 @@ attn_status launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUten
                        void* o, float* lse, const Problem& p, cudaStream_t stream) {
   using Cfg = attn::FwdCfg<D>;
   auto kern = attn::fwd_kernel<D, MODE, FEAT>;
-  static std::once_flag attr_once;
-  static cudaError_t attr_err = cudaSuccess;
-  static int launch_regs = 0;
-  std::call_once(attr_once, [&] {
-    attr_err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                    Cfg::kSmemAlloc);
-    cudaFuncAttributes fa;
-    if (attr_err == cudaSuccess) attr_err = cudaFuncGetAttributes(&fa, kern);
-    if (attr_err == cudaSuccess) launch_regs = fa.numRegs;
-  });
+  static KernelSetup setup;
+  int launch_regs = 0;
+  const cudaError_t attr_err = prepare_kernel(kern, Cfg::kSmemAlloc, setup, &launch_regs);
   if (attr_err != cudaSuccess) return cuda_fail(attr_err, "cudaFuncSetAttribute(fwd)");
   // The kernel rebalances registers between warpgroups with setmaxnreg; that
   // split is only valid for the launch register count it was written for.
@@ -264,15 +315,6 @@ attn_status launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUten
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "fwd kernel launch");
   return ATTN_OK;
-}
-
-// One-time per-kernel setup: opt in to the dynamic shared memory size.
-template <typename Kern>
-cudaError_t set_smem_once(Kern kern, int bytes, std::once_flag& once, cudaError_t& err) {
-  std::call_once(once, [&] {
-    err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
-  });
-  return err;
 }
 
 struct BwdArgs {
@@ -304,13 +346,12 @@ attn_status launch_bwd(const BwdArgs& a, const Problem& p, cudaStream_t stream) 
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "bwd preprocess launch");
 
-  static std::once_flag o1, o2;
-  static cudaError_t e1 = cudaSuccess, e2 = cudaSuccess;
+  static KernelSetup s1, s2;
   auto k1 = bwd_dkdv_kernel<D, MODE, FEAT>;
   auto k2 = bwd_dq_kernel<D, MODE, FEAT>;
-  if ((e = set_smem_once(k1, DkdvCfg<D>::kSmemAlloc, o1, e1)) != cudaSuccess)
+  if ((e = prepare_kernel(k1, DkdvCfg<D>::kSmemAlloc, s1)) != cudaSuccess)
     return cuda_fail(e, "cudaFuncSetAttribute(dkdv)");
-  if ((e = set_smem_once(k2, DqCfg<D>::kSmemAlloc, o2, e2)) != cudaSuccess)
+  if ((e = prepare_kernel(k2, DqCfg<D>::kSmemAlloc, s2)) != cudaSuccess)
     return cuda_fail(e, "cudaFuncSetAttribute(dq)");
 
   ProfScope p1(kProfBwdDkdv, stream);
@@ -356,7 +397,6 @@ __global__ void selftest_wait_timeout_kernel() {
 constexpr size_t kStaticScratchBytes = size_t(8) << 20;
 static __device__ __align__(256) float g_bwd_scratch[kStaticScratchBytes / sizeof(float)];
 
-constexpr int kMaxDevices = 64;
 std::mutex g_scratch_mu;
 void* g_scratch_addr[kMaxDevices] = {};
 
@@ -502,19 +542,9 @@ attn_status check_offsets_args(const int* cu_q, const int* cu_k) {
 }
 
 attn_status check_offsets(const int* cu_q, const int* cu_k) {
-  const void* ptrs[2] = {cu_q, cu_k};
-  const char* names[2] = {"cu_seqlens_q", "cu_seqlens_k"};
-  for (int i = 0; i < 2; ++i) {
-    cudaPointerAttributes pa;
-    cudaError_t e = cudaPointerGetAttributes(&pa, ptrs[i]);
-    if (e != cudaSuccess) {
-      cudaGetLastError();
-      return fail(ATTN_ERR_ARG, "%s is not a CUDA pointer (%s)", names[i], cudaGetErrorName(e));
-    }
-    if (pa.type != cudaMemoryTypeDevice && pa.type != cudaMemoryTypeManaged)
-      return fail(ATTN_ERR_ARG, "%s is not device memory", names[i]);
-  }
-  return ATTN_OK;
+  attn_status st = check_device_ptr(cu_q, "cu_seqlens_q");
+  if (st != ATTN_OK) return st;
+  return check_device_ptr(cu_k, "cu_seqlens_k");
 }
 
 // Packed-batch argument checks (host side; offsets are checked on the GPU).
