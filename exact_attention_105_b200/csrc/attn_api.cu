@@ -103,6 +103,13 @@ std::once_flag g_init_once;
 
 // Devices a process may use (per-device caches below are indexed by ordinal).
 constexpr int kMaxDevices = 64;
+int g_sm_count[kMaxDevices] = {};             // multiprocessors, filled by check_device()
+
+int sm_count() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 148;
+  return g_sm_count[dev] > 0 ? g_sm_count[dev] : 148;
+}
 
 void init_once() {
   cudaDriverEntryPointQueryResult q;
@@ -137,6 +144,7 @@ attn_status check_device() {
       return fail(ATTN_ERR_CUDA, "cudaGetDeviceProperties(%d): %s", dev, cudaGetErrorString(e));
     }
     arch[dev] = prop.major * 10 + prop.minor;
+    g_sm_count[dev] = prop.multiProcessorCount;
   }
   if (arch[dev] != 100)
     return fail(ATTN_ERR_CUDA, "this library is built for sm_100a (B200); device %d is sm_%d", dev,
@@ -303,14 +311,19 @@ attn_status launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUten
   if (launch_regs != attn::kFwdRegsLaunch)
     return fail(ATTN_ERR_CUDA, "fwd kernel built with %d registers/thread, expected %d",
                 launch_regs, attn::kFwdRegsLaunch);
-  const long long blocks = static_cast<long long>(p.B) * p.Hq * ((p.geom.Nq + 255) / 256);
+  // Two 128-row tiles per CTA share each K/V tile; when that leaves SMs idle,
+  // one tile per CTA doubles the CTAs.
+  const long long pairs = static_cast<long long>(p.B) * p.Hq * ((p.geom.Nq + 255) / 256);
+  const int one_tile = pairs < sm_count() ? 1 : 0;
+  const long long blocks = one_tile ? static_cast<long long>(p.B) * p.Hq * ((p.geom.Nq + 127) / 128)
+                                    : pairs;
   if (blocks > 0x7FFFFFFFLL) return fail(ATTN_ERR_ARG, "problem too large for one launch");
   dim3 grid(static_cast<unsigned>(blocks));
   const float scale_log2 = p.scale * 1.4426950408889634f;
   ProfScope ps(kProfFwd, stream);
   kern<<<grid, Cfg::kThreads, Cfg::kSmemAlloc, stream>>>(
       mq, mk, mv, static_cast<__nv_bfloat16*>(o), lse, p.Hq, p.Hq / p.Hkv, p.geom, scale_log2,
-      p.mask.win, p.cap);
+      p.mask.win, p.cap, one_tile);
   ps.end();
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "fwd kernel launch");

@@ -81,7 +81,7 @@ __global__ void __launch_bounds__(384, 1)
 fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
            const __grid_constant__ CUtensorMap tm_v, __nv_bfloat16* __restrict__ out,
            float* __restrict__ lse_out, int Hq, int group, SeqGeom geom, float scale_log2,
-           KeyWindow win, Softcap cap) {
+           KeyWindow win, Softcap cap, int one_tile) {
   constexpr bool SOFTCAP = (FEAT & kFeatSoftcap) != 0;
   constexpr bool PACKED = (FEAT & kFeatPacked) != 0;
   static_assert(FEAT == 0 || MODE == kMaskGeneral, "features run in the general mode");
@@ -107,7 +107,10 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
   // 1-D grid, (batch, query head) fastest, then 256-row query block from the
   // last (heaviest when causal) to the first: every head's heaviest block is
   // dispatched before any lighter one, which keeps the causal tail short.
-  const int nmb = (geom.Nq + 255) >> 8;
+  // Rows per CTA: two 128-row tiles, or one when the problem is too small to
+  // fill the GPU with two-tile CTAs (more CTAs, one tile each).
+  const int rb = one_tile ? 128 : 256;
+  const int nmb = (geom.Nq + rb - 1) / rb;
   const int BH = gridDim.x / nmb;
   const int bh = blockIdx.x % BH;                  // b * Hq + hq
   const int b = bh / Hq;
@@ -115,7 +118,8 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
   const int mb = nmb - 1 - static_cast<int>(blockIdx.x / BH);
   const SeqSpan sp = seq_span<PACKED>(geom, b);
   const int Nq = sp.nq, Nk = sp.nk;
-  if (mb * 256 >= Nq) return;                      // packed batch: past this sequence's rows
+  const int m0 = mb * rb;                          // first query row of this CTA
+  if (m0 >= Nq) return;                            // packed batch: past this sequence's rows
   win.off = Nk - Nq;                               // bottom-right alignment per sequence
   // TMA z coordinates of the query head and its KV head (GQA: contiguous groups).
   const int zq = PACKED ? hq : bh;
@@ -129,9 +133,9 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
   // tile number: that would live in local memory and be reloaded after every
   // barrier wait on the MMA issue path.
   int lo0 = 0, hi0 = -1, lo1 = 0, hi1 = -1;
-  if (mb * 256 < Nq) kv_tile_range<MODE>(mb * 256, min(mb * 256 + 127, Nq - 1), Nk, win, lo0, hi0);
-  if (mb * 256 + 128 < Nq)
-    kv_tile_range<MODE>(mb * 256 + 128, min(mb * 256 + 255, Nq - 1), Nk, win, lo1, hi1);
+  kv_tile_range<MODE>(m0, min(m0 + 127, Nq - 1), Nk, win, lo0, hi0);
+  if (!one_tile && m0 + 128 < Nq)
+    kv_tile_range<MODE>(m0 + 128, min(m0 + 255, Nq - 1), Nk, win, lo1, hi1);
   const int n0 = max(0, hi0 - lo0 + 1), n1 = max(0, hi1 - lo1 + 1);
   auto lo_t = [&](int t) { return t ? lo1 : lo0; };
   auto hi_t = [&](int t) { return t ? hi1 : hi0; };
@@ -179,7 +183,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
 #pragma unroll
           for (int a = 0; a < D / 64; ++a)
             tma_load_3d(smem + C::kQOff + t * C::kTileBytes + a * 16384, &tm_q, &q_full[t],
-                        a * 64, sp.q0 + mb * 256 + t * 128, zq);
+                        a * 64, sp.q0 + m0 + t * 128, zq);
         }
       }
       uint32_t issued = 0;
@@ -300,13 +304,13 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
     regs_grow<kFwdRegsSoftmax>();
     const int t = warp >> 2;
     const int quad = warp & 3;
-    const int row = mb * 256 + t * 128 + quad * 32 + lane;
+    const int row = m0 + t * 128 + quad * 32 + lane;
     const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
     const uint32_t t_s = tmem + lane_base + t * 128;
     const uint32_t t_p = t_s + 64;
     const uint32_t t_o = tmem + lane_base + 256 + t * 128;
     const int n = n_t(t);
-    const int r_first = mb * 256 + t * 128;                  // first and last row of this tile
+    const int r_first = m0 + t * 128;                        // first and last row of this tile
     const int r_last = min(r_first + 127, Nq - 1);
     // Visible keys of this row: [k_lo, k_hi] (k_hi < k_lo: none).
     const int k_lo = (MODE == kMaskGeneral) ? max(0, win.lo(row)) : 0;
@@ -448,7 +452,8 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
     }
 
     // Epilogue. A row that saw no key (l = 0) gets O = 0 and lse = -inf.
-    const bool present = r_first < Nq;
+    // Tile 1 of a one-tile CTA holds rows of the next CTA: never write them.
+    const bool present = r_first < Nq && (t == 0 || !one_tile);
     if (ok) ok = mbar_wait(&o_full[t], 0, abort_flag, kSiteOFull);
     if (ok || (present && n == 0)) {
       const bool has_o = n > 0;
