@@ -628,7 +628,8 @@ def run_ours(args):
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline and not fwd_only:
         cpu = oracle_baseline(w, host, steps=3, per_step_s=4.0)
-        cpu = {k2: cpu[k2] for k2 in ("value", "unit", "cores", "kind", "sample")}
+        cpu = {k2: cpu[k2] for k2 in ("value", "unit", "cores", "kind", "sample", "seconds",
+                                    "gflops", "blas")}
 
     if world > 1:
         dist.barrier()
