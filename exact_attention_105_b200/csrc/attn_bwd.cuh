@@ -21,8 +21,14 @@
 //                    when causal). Per block it computes S^T, dP^T, P^T, dS^T
 //                    and accumulates dV and dK in TMEM.
 //   bwd_dq_kernel    one CTA per (batch, query head, 128-query block). Q_i and
-//                    dO_i stay resident while K_j/V_j stream through a ring. Per
-//                    block it computes S, dP, P, dS and accumulates dQ in TMEM.
+//                    dO_i stay resident while K_j and V_j stream through two
+//                    rings (K_j is held from S(j) to dQ(j), V_j only for dP(j)).
+//                    Per key block it computes S, dP, P, dS and accumulates dQ
+//                    in TMEM: S in columns [0, 128), dQ in [256, 384), and dP
+//                    of block j, overwritten by its dS, in [128, 256) for even
+//                    j and [384, 512) for odd j. With two dP buffers, dP(j+1)
+//                    is issued right after S(j+1), ahead of dQ(j), and waits
+//                    only for dQ(j-1), which read the same buffer.
 // Warp roles in both main kernels (384 threads): warps 0-7 are two compute
 // warpgroups, warp 8 is the TMA producer, warp 9 allocates TMEM and issues
 // the MMAs, and warps 10-11 idle. Thread r of a compute warpgroup owns TMEM
@@ -425,8 +431,7 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       };
       p_block(r0, 0);
       p_block(r1, 32);
-      tmem_st16(t_s, &pw[0]);
-      tmem_st16(t_s + 16, &pw[16]);
+      tmem_st32(t_s, pw);
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(p_full);
@@ -438,13 +443,12 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       tmem_ld32(t_dp + 32, d1);
       tmem_ld_wait(d0);
       reg_fence(d1);
-      uint32_t ds[16];
+      uint32_t ds[32];
       ds_block(&pf[0], d0, ds,
                [&](int e) { return *reinterpret_cast<const float2*>(&Ds[e]); });
-      tmem_st16(t_dp, ds);
-      ds_block(&pf[32], d1, ds,
+      ds_block(&pf[32], d1, ds + 16,
                [&](int e) { return *reinterpret_cast<const float2*>(&Ds[32 + e]); });
-      tmem_st16(t_dp + 16, ds);
+      tmem_st32(t_dp, ds);
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(ds_full);
@@ -482,13 +486,16 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 template <int D>
 struct DqCfg {
   static constexpr int kTile = 128 * D * 2;
-  static constexpr int kStages = (D == 128) ? 4 : 6;     // K/V ring slots
+  static constexpr int kKStages = 3;                     // K ring: K_j lives from S(j) to dQ(j)
+  static constexpr int kVStages = (D == 128) ? 2 : 3;    // V ring: V_j lives for dP(j) only
   static constexpr int kQOff = 0;
   static constexpr int kDOOff = kTile;
-  static constexpr int kKVOff = 2 * kTile;
-  static constexpr int kBarOff = kKVOff + kStages * kTile;
-  // qd_full kv_full[S] kv_empty[S] s_full s_free dp_full ds_full acc_done mma_done
-  static constexpr int kNumBars = 1 + 2 * kStages + 6;
+  static constexpr int kKOff = 2 * kTile;
+  static constexpr int kVOff = kKOff + kKStages * kTile;
+  static constexpr int kBarOff = kVOff + kVStages * kTile;
+  // qd_full k_full[KS] k_empty[KS] v_full[VS] v_empty[VS] s_full s_free dp_full[2] ds_full[2]
+  // acc_done mma_done
+  static constexpr int kNumBars = 1 + 2 * kKStages + 2 * kVStages + 8;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
   static constexpr int kBytes = kMiscOff + 16;
   static constexpr int kSmemAlloc = kBytes + 1024;
@@ -506,19 +513,21 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
   constexpr bool PACKED = (FEAT & kFeatPacked) != 0;
   static_assert(FEAT == 0 || MODE == kMaskGeneral, "features run in the general mode");
   using C = DqCfg<D>;
-  constexpr int NS = C::kStages;
+  constexpr int KS = C::kKStages, VS = C::kVStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   const uint32_t sbase = smem_u32(smem);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kBarOff);
   uint64_t* qd_full = bars;
-  uint64_t* kv_full = qd_full + 1;
-  uint64_t* kv_empty = kv_full + NS;
-  uint64_t* s_full = kv_empty + NS;
+  uint64_t* k_full = qd_full + 1;
+  uint64_t* k_empty = k_full + KS;
+  uint64_t* v_full = k_empty + KS;
+  uint64_t* v_empty = v_full + VS;
+  uint64_t* s_full = v_empty + VS;
   uint64_t* s_free = s_full + 1;
-  uint64_t* dp_full = s_free + 1;
-  uint64_t* ds_full = dp_full + 1;
-  uint64_t* acc_done = ds_full + 1;
+  uint64_t* dp_full = s_free + 1;            // [2]: dP buffer b holds a new step
+  uint64_t* ds_full = dp_full + 2;           // [2]: dS written into buffer b
+  uint64_t* acc_done = ds_full + 2;
   uint64_t* mma_done = acc_done + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kMiscOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kMiscOff + 4);
@@ -543,14 +552,20 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
 
   if (threadIdx.x == 0) {
     mbar_init(qd_full, 1);
-    for (int s = 0; s < NS; ++s) {
-      mbar_init(&kv_full[s], 1);
-      mbar_init(&kv_empty[s], 1);
+    for (int s = 0; s < KS; ++s) {
+      mbar_init(&k_full[s], 1);
+      mbar_init(&k_empty[s], 1);
+    }
+    for (int s = 0; s < VS; ++s) {
+      mbar_init(&v_full[s], 1);
+      mbar_init(&v_empty[s], 1);
     }
     mbar_init(s_full, 1);
     mbar_init(s_free, 256);
-    mbar_init(dp_full, 1);
-    mbar_init(ds_full, 256);
+    for (int b2 = 0; b2 < 2; ++b2) {
+      mbar_init(&dp_full[b2], 1);
+      mbar_init(&ds_full[b2], 256);
+    }
     mbar_init(acc_done, 1);
     mbar_init(mma_done, 1);
     *abort_flag = 0;
@@ -580,36 +595,50 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
           tma_load_3d(smem + C::kDOOff + a * 16384, &tm_do, qd_full, a * 64, sp.q0 + i * 128, zq);
         }
       }
-      uint32_t issued = 0;
-      bool ok = true;
-      for (int jj = 0; jj < n && ok; ++jj) {
-        for (int w = 0; w < 2; ++w) {
-          const uint32_t s = issued % NS, round = issued / NS;
-          if (round > 0 && !mbar_wait(&kv_empty[s], (round - 1) & 1u, abort_flag, kSiteBLoadEmpty)) {
-            ok = false;
-            break;
-          }
-          mbar_expect_tx(&kv_full[s], C::kTile);
+      int issued_k = 0, issued_v = 0;
+      // One ring per operand: K_j, then V_j, each into its own ring.
+      auto load = [&](int jj, bool is_v) {
+        const int ns = is_v ? VS : KS;
+        const int s = jj % ns, round = jj / ns;
+        uint64_t* full = is_v ? &v_full[s] : &k_full[s];
+        uint64_t* empty = is_v ? &v_empty[s] : &k_empty[s];
+        if (round > 0 && !mbar_wait(empty, (round - 1) & 1u, abort_flag, kSiteBLoadEmpty))
+          return false;
+        mbar_expect_tx(full, C::kTile);
+        uint8_t* dst = smem + (is_v ? C::kVOff : C::kKOff) + s * C::kTile;
 #pragma unroll
-          for (int a = 0; a < D / 64; ++a)
-            tma_load_3d(smem + C::kKVOff + s * C::kTile + a * 16384, w ? &tm_v : &tm_k, &kv_full[s],
-                        a * 64, sp.k0 + (j_lo + jj) * 128, zkv);
-          ++issued;
-        }
+        for (int a = 0; a < D / 64; ++a)
+          tma_load_3d(dst + a * 16384, is_v ? &tm_v : &tm_k, full, a * 64,
+                      sp.k0 + (j_lo + jj) * 128, zkv);
+        return true;
+      };
+      for (int jj = 0; jj < n; ++jj) {
+        if (!load(jj, false)) break;
+        ++issued_k;
+        if (!load(jj, true)) break;
+        ++issued_v;
       }
       if (n > 0) mbar_wait_drain(qd_full, 0);
-      const uint32_t first = issued > (uint32_t)NS ? issued - NS : 0u;
-      for (uint32_t x = first; x < issued; ++x) mbar_wait_drain(&kv_full[x % NS], (x / NS) & 1u);
+      for (int x = max(0, issued_k - KS); x < issued_k; ++x)
+        mbar_wait_drain(&k_full[x % KS], (x / KS) & 1);
+      for (int x = max(0, issued_v - VS); x < issued_v; ++x)
+        mbar_wait_drain(&v_full[x % VS], (x / VS) & 1);
     }
   } else if (warp == 9) {
     if (lane == 0) {
       // -------------------------------------------------------- MMA issuer
       constexpr uint32_t kIdescSS = idesc_bf16_f32(128, 128, 0, 0);
       constexpr uint32_t kIdescAcc = idesc_bf16_f32(128, D, 0, 1);
-      auto slot = [&](uint32_t idx) { return sbase + C::kKVOff + (idx % NS) * C::kTile; };
-      auto kv_wait = [&](uint32_t idx) {
-        return mbar_wait(&kv_full[idx % NS], (idx / NS) & 1u, abort_flag, kSiteBKV);
+      auto kslot = [&](int jj) { return sbase + C::kKOff + (jj % KS) * C::kTile; };
+      auto vslot = [&](int jj) { return sbase + C::kVOff + (jj % VS) * C::kTile; };
+      auto k_wait = [&](int jj) {
+        return mbar_wait(&k_full[jj % KS], (jj / KS) & 1, abort_flag, kSiteBKV);
       };
+      auto v_wait = [&](int jj) {
+        return mbar_wait(&v_full[jj % VS], (jj / VS) & 1, abort_flag, kSiteBKV);
+      };
+      // dP / dS of step jj live in TMEM columns [128, 256) (even jj) or [384, 512) (odd jj).
+      auto dp_col = [&](int jj) { return (jj & 1) ? 384u : 128u; };
       auto mma_tile_kk = [&](uint32_t dst, uint32_t a, uint32_t bt) {
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
@@ -618,45 +647,47 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                  kk > 0 ? 1u : 0u);
         }
       };
-      bool ok = n > 0 && mbar_wait(qd_full, 0, abort_flag, kSiteBLoadFull) && kv_wait(0);
+      bool ok = n > 0 && mbar_wait(qd_full, 0, abort_flag, kSiteBLoadFull) && k_wait(0);
       if (ok) {
         tc_fence_after();
-        mma_tile_kk(tmem + 0, sbase + C::kQOff, slot(0));        // S(0) = Q K_0^T
+        mma_tile_kk(tmem + 0, sbase + C::kQOff, kslot(0));            // S(0) = Q K_0^T
         tc_commit(s_full);
-        ok = kv_wait(1);
+        ok = v_wait(0);
       }
       if (ok) {
         tc_fence_after();
-        mma_tile_kk(tmem + 128, sbase + C::kDOOff, slot(1));     // dP(0) = dO V_0^T
-        tc_commit(dp_full);
+        mma_tile_kk(tmem + dp_col(0), sbase + C::kDOOff, vslot(0));   // dP(0) = dO V_0^T
+        tc_commit(&dp_full[0]);
+        tc_commit(&v_empty[0]);
       }
       for (int jj = 0; ok && jj < n; ++jj) {
-        const uint32_t ik = 2 * jj, iv = 2 * jj + 1;
         const bool more = jj + 1 < n;
         if (more) {
-          if (!mbar_wait(s_free, jj & 1, abort_flag, kSiteBSFree) || !kv_wait(ik + 2)) {
+          // S(j+1) once S(j) is in registers; dP(j+1) into the buffer dQ(j-1) has read.
+          if (!mbar_wait(s_free, jj & 1, abort_flag, kSiteBSFree) || !k_wait(jj + 1)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          mma_tile_kk(tmem + 0, sbase + C::kQOff, slot(ik + 2));  // S(j+1)
+          mma_tile_kk(tmem + 0, sbase + C::kQOff, kslot(jj + 1));
           tc_commit(s_full);
-        }
-        if (!mbar_wait(ds_full, jj & 1, abort_flag, kSiteBDS)) { ok = false; break; }
-        tc_fence_after();
-        const uint32_t kb = slot(ik);
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk)                           // dQ += dS K_j
-          mma_ts(tmem + 256, tmem + 128 + split_col(kk), sdesc_sw128(kb + kk * 2048, 16384, 1024),
-                 kIdescAcc, (jj > 0 || kk > 0) ? 1u : 0u);
-        tc_commit(&kv_empty[ik % NS]);
-        tc_commit(&kv_empty[iv % NS]);
-        if (more) {
-          if (!kv_wait(iv + 2)) { ok = false; break; }
+          if (!v_wait(jj + 1)) { ok = false; break; }
           tc_fence_after();
-          mma_tile_kk(tmem + 128, sbase + C::kDOOff, slot(iv + 2)); // dP(j+1)
-          tc_commit(dp_full);
+          mma_tile_kk(tmem + dp_col(jj + 1), sbase + C::kDOOff, vslot(jj + 1));
+          tc_commit(&dp_full[(jj + 1) & 1]);
+          tc_commit(&v_empty[(jj + 1) % VS]);
         }
+        if (!mbar_wait(&ds_full[jj & 1], (jj >> 1) & 1, abort_flag, kSiteBDS)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t kb = kslot(jj);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)                                // dQ += dS K_j
+          mma_ts(tmem + 256, tmem + dp_col(jj) + split_col(kk),
+                 sdesc_sw128(kb + kk * 2048, 16384, 1024), kIdescAcc, (jj > 0 || kk > 0) ? 1u : 0u);
+        tc_commit(&k_empty[jj % KS]);
       }
       if (ok) tc_commit(acc_done);
       if (n > 0) {                           // nothing to drain when nothing was issued
@@ -678,7 +709,7 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                                             : ((MODE == kMaskCausal) ? min(row, Nk - 1) : Nk - 1);
     const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
     const uint32_t t_s = tmem + lane_base + 64 * h;
-    const uint32_t t_dp = tmem + lane_base + 128 + 64 * h;   // dP half; dS into +0..32
+    const uint32_t t_dp0 = tmem + lane_base + 128 + 64 * h;  // dP half of buffer 0; dS into +0..32
     const int c_base = 64 * h;
     const size_t ws = static_cast<size_t>(bh) * Npad + row;   // row < Npad always
     const float nLr = Lws[ws];                                // -lse*log2e; -inf on padding rows
@@ -738,23 +769,24 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
       p_block(r0, 0);
       p_block(r1, 32);
 
-      if (!mbar_wait(dp_full, jj & 1, abort_flag, kSiteBDP)) { ok = false; break; }
+      // dP(j) and dS(j) use buffer j & 1 (TMEM columns 128.. or 384..).
+      const uint32_t t_dp = t_dp0 + (jj & 1) * 256;
+      if (!mbar_wait(&dp_full[jj & 1], (jj >> 1) & 1, abort_flag, kSiteBDP)) { ok = false; break; }
       tc_fence_after();
       uint32_t d0[32], d1[32];
       tmem_ld32(t_dp, d0);
       tmem_ld32(t_dp + 32, d1);
       tmem_ld_wait(d0);
       reg_fence(d1);
-      uint32_t ds[16];
+      uint32_t ds[32];
       const float2 nd2 = make_float2(nDr, nDr);
       auto nd = [&](int) { return nd2; };
       ds_block(&pf[0], d0, ds, nd);
-      tmem_st16(t_dp, ds);
-      ds_block(&pf[32], d1, ds, nd);
-      tmem_st16(t_dp + 16, ds);
+      ds_block(&pf[32], d1, ds + 16, nd);
+      tmem_st32(t_dp, ds);
       tmem_st_wait();
       tc_fence_before();
-      mbar_arrive(ds_full);
+      mbar_arrive(&ds_full[jj & 1]);
     }
     if (ok && n > 0) ok = mbar_wait(acc_done, 0, abort_flag, kSiteBAcc);
     if (ok) {
