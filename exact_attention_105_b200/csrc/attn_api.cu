@@ -193,7 +193,8 @@ cudaError_t prepare_kernel(Kern kern, int smem_bytes, KernelSetup& ks, int* regs
 // (one 128-row, 128-byte-wide column block) and 128-byte swizzle. Row and z
 // strides are in elements. Fixed-length [B*H, N, d]: rows = N, z = B*H,
 // row stride d, z stride N*d. Packed [total, H, d]: rows = total, z = H, row
-// stride H*d, z stride d. Rows past `rows` read as zeros.
+// stride H*d, z stride d. Rows past `rows` read as zeros, and stores to them
+// are dropped.
 attn_status make_map(CUtensorMap* map, const void* base, int d, long long rows, long long zdim,
                      long long row_stride, long long z_stride) {
   cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(rows),
@@ -299,7 +300,8 @@ struct Problem {
 
 template <int D, int MODE, int FEAT>
 attn_status launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
-                       void* o, float* lse, const Problem& p, cudaStream_t stream) {
+                       const CUtensorMap& mo, void* o, float* lse, const Problem& p,
+                       cudaStream_t stream) {
   using Cfg = attn::FwdCfg<D>;
   auto kern = attn::fwd_kernel<D, MODE, FEAT>;
   static KernelSetup setup;
@@ -322,7 +324,7 @@ attn_status launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUten
   const float scale_log2 = p.scale * 1.4426950408889634f;
   ProfScope ps(kProfFwd, stream);
   kern<<<grid, Cfg::kThreads, Cfg::kSmemAlloc, stream>>>(
-      mq, mk, mv, static_cast<__nv_bfloat16*>(o), lse, p.Hq, p.Hq / p.Hkv, p.geom, scale_log2,
+      mq, mk, mv, mo, static_cast<__nv_bfloat16*>(o), lse, p.Hq, p.Hq / p.Hkv, p.geom, scale_log2,
       p.mask.win, p.cap, one_tile);
   ps.end();
   cudaError_t e = cudaGetLastError();
@@ -331,7 +333,7 @@ attn_status launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUten
 }
 
 struct BwdArgs {
-  CUtensorMap mq, mk, mv, mdo;
+  CUtensorMap mq, mk, mv, mdo, mdk, mdv, mdq;
   const void* o;
   const float* lse;
   const void* dO;
@@ -369,15 +371,15 @@ attn_status launch_bwd(const BwdArgs& a, const Problem& p, cudaStream_t stream) 
 
   ProfScope p1(kProfBwdDkdv, stream);
   k1<<<dim3(static_cast<unsigned>(g1)), DkdvCfg<D>::kThreads, DkdvCfg<D>::kSmemAlloc, stream>>>(
-      a.mq, a.mk, a.mv, a.mdo, a.L, a.Dv, static_cast<__nv_bfloat16*>(a.dk),
+      a.mq, a.mk, a.mv, a.mdo, a.mdk, a.mdv, a.L, a.Dv, static_cast<__nv_bfloat16*>(a.dk),
       static_cast<__nv_bfloat16*>(a.dv), p.Hq, group, p.geom, Npad, scale_log2, p.scale,
       p.mask.win, p.cap);
   p1.end();
   if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "bwd dK/dV launch");
   ProfScope p2(kProfBwdDq, stream);
   k2<<<dim3(static_cast<unsigned>(g2)), DqCfg<D>::kThreads, DqCfg<D>::kSmemAlloc, stream>>>(
-      a.mq, a.mk, a.mv, a.mdo, a.L, a.Dv, static_cast<__nv_bfloat16*>(a.dq), p.Hq, group, p.geom,
-      Npad, scale_log2, p.scale, p.mask.win, p.cap);
+      a.mq, a.mk, a.mv, a.mdo, a.mdq, a.L, a.Dv, static_cast<__nv_bfloat16*>(a.dq), p.Hq, group,
+      p.geom, Npad, scale_log2, p.scale, p.mask.win, p.cap);
   p2.end();
   if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "bwd dQ launch");
   return ATTN_OK;
@@ -442,18 +444,21 @@ __global__ void fill_neg_inf_kernel(float* p, long long n) {
 
 template <int D>
 attn_status dispatch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                         const CUtensorMap& mo,
                          void* o, float* lse, const Problem& p, cudaStream_t stream) {
   using namespace attn;
-  if (p.mask.mode == kMaskNone) return launch_fwd<D, kMaskNone, 0>(mq, mk, mv, o, lse, p, stream);
+  if (p.mask.mode == kMaskNone)
+    return launch_fwd<D, kMaskNone, 0>(mq, mk, mv, mo, o, lse, p, stream);
   if (p.mask.mode == kMaskCausal)
-    return launch_fwd<D, kMaskCausal, 0>(mq, mk, mv, o, lse, p, stream);
+    return launch_fwd<D, kMaskCausal, 0>(mq, mk, mv, mo, o, lse, p, stream);
   const bool packed = p.geom.cu_q != nullptr;
   if (packed && p.mask.softcap)
-    return launch_fwd<D, kMaskGeneral, kFeatPacked | kFeatSoftcap>(mq, mk, mv, o, lse, p, stream);
-  if (packed) return launch_fwd<D, kMaskGeneral, kFeatPacked>(mq, mk, mv, o, lse, p, stream);
+    return launch_fwd<D, kMaskGeneral, kFeatPacked | kFeatSoftcap>(mq, mk, mv, mo, o, lse, p,
+                                                                    stream);
+  if (packed) return launch_fwd<D, kMaskGeneral, kFeatPacked>(mq, mk, mv, mo, o, lse, p, stream);
   if (p.mask.softcap)
-    return launch_fwd<D, kMaskGeneral, kFeatSoftcap>(mq, mk, mv, o, lse, p, stream);
-  return launch_fwd<D, kMaskGeneral, 0>(mq, mk, mv, o, lse, p, stream);
+    return launch_fwd<D, kMaskGeneral, kFeatSoftcap>(mq, mk, mv, mo, o, lse, p, stream);
+  return launch_fwd<D, kMaskGeneral, 0>(mq, mk, mv, mo, o, lse, p, stream);
 }
 
 template <int D>
@@ -602,12 +607,13 @@ attn_status fwd_run(const void* q, const void* k, const void* v, void* o, float*
     if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "lse fill launch");
     return ATTN_OK;
   }
-  CUtensorMap mq, mk, mv;
+  CUtensorMap mq, mk, mv, mo;
   if ((st = make_map(&mq, q, p.d, L.q_rows, L.q_z, L.q_rs, L.q_zs)) != ATTN_OK) return st;
+  if ((st = make_map(&mo, o, p.d, L.q_rows, L.q_z, L.q_rs, L.q_zs)) != ATTN_OK) return st;
   if ((st = make_map(&mk, k, p.d, L.k_rows, L.k_z, L.k_rs, L.k_zs)) != ATTN_OK) return st;
   if ((st = make_map(&mv, v, p.d, L.k_rows, L.k_z, L.k_rs, L.k_zs)) != ATTN_OK) return st;
-  if (p.d == 64) return dispatch_fwd<64>(mq, mk, mv, o, lse, p, stream);
-  return dispatch_fwd<128>(mq, mk, mv, o, lse, p, stream);
+  if (p.d == 64) return dispatch_fwd<64>(mq, mk, mv, mo, o, lse, p, stream);
+  return dispatch_fwd<128>(mq, mk, mv, mo, o, lse, p, stream);
 }
 
 // Backward shared by every backward entry point. With use_static the scratch
@@ -656,6 +662,9 @@ attn_status bwd_run(const void* q, const void* k, const void* v, const void* o,
   if ((st = make_map(&a.mk, k, p.d, L.k_rows, L.k_z, L.k_rs, L.k_zs)) != ATTN_OK) return st;
   if ((st = make_map(&a.mv, v, p.d, L.k_rows, L.k_z, L.k_rs, L.k_zs)) != ATTN_OK) return st;
   if ((st = make_map(&a.mdo, dO, p.d, L.q_rows, L.q_z, L.q_rs, L.q_zs)) != ATTN_OK) return st;
+  if ((st = make_map(&a.mdk, dk, p.d, L.k_rows, L.k_z, L.k_rs, L.k_zs)) != ATTN_OK) return st;
+  if ((st = make_map(&a.mdv, dv, p.d, L.k_rows, L.k_z, L.k_rs, L.k_zs)) != ATTN_OK) return st;
+  if ((st = make_map(&a.mdq, dq, p.d, L.q_rows, L.q_z, L.q_rs, L.q_zs)) != ATTN_OK) return st;
   // The preprocess kernel writes every scratch row the other two kernels
   // read, so nothing left from an earlier call is ever used and no clearing
   // is needed (this matters for the static area).

@@ -37,6 +37,11 @@
 // 64 columns, so neither group overwrites columns the other has yet to read.
 // The MMA that consumes them reads K-step kk (16 columns) from TMEM column
 // 64*(kk/4) + 8*(kk%4) of the tile.
+// Both kernels end by staging their bf16 output tile (dK and dV, or dQ) in
+// shared memory that no MMA reads any more (the K/V tiles, or the Q tile),
+// 128-byte swizzled, and writing it with TMA stores. Packed tiles that run
+// past their sequence are written row by row instead, since the tensor map
+// only bounds the whole packed tensor.
 #pragma once
 
 #include "geometry.cuh"
@@ -156,6 +161,30 @@ __device__ __forceinline__ void store_acc_row(uint32_t t_acc, __nv_bfloat16* dst
   }
 }
 
+// Epilogue helper: this thread's 128 x D fp32 accumulator row (tile row t)
+// -> bf16 * mul into a shared-memory tile laid out as the 128-byte-swizzled
+// TMA box expects: D/64 blocks of 128 rows x 128 bytes, the 16-byte chunk c
+// of row t at chunk position c ^ (t & 7).
+template <int D, int C0 = 0, int C1 = D / 32>
+__device__ __forceinline__ void stage_acc_row(uint32_t t_acc, uint8_t* tile, int t, float mul) {
+#pragma unroll
+  for (int cc = C0; cc < C1; ++cc) {
+    uint32_t a[32];
+    tmem_ld32(t_acc + cc * 32, a);
+    tmem_ld_wait(a);
+    uint32_t pk[16];
+#pragma unroll
+    for (int e = 0; e < 16; ++e) pk[e] = pack_bf16x2(u2f(a[2 * e]) * mul, u2f(a[2 * e + 1]) * mul);
+    uint8_t* rowp = tile + (cc >> 1) * 16384 + t * 128;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int c = (cc & 1) * 4 + q;
+      *reinterpret_cast<uint4*>(rowp + ((c ^ (t & 7)) << 4)) =
+          make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
+    }
+  }
+}
+
 // ------------------------------------------------------------------ dK / dV
 template <int D>
 struct DkdvCfg {
@@ -178,6 +207,8 @@ template <int D, int MODE, int FEAT>
 __global__ void __launch_bounds__(384, 1)
 bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+                const __grid_constant__ CUtensorMap tm_dk,
+                const __grid_constant__ CUtensorMap tm_dv,
                 const float* __restrict__ Lws, const float* __restrict__ Dws,
                 __nv_bfloat16* __restrict__ dk, __nv_bfloat16* __restrict__ dv, int Hq, int group,
                 SeqGeom geom, int Npad, float scale_log2, float scale, KeyWindow win,
@@ -454,7 +485,30 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       mbar_arrive(ds_full);
     }
     if (ok && n_steps > 0) ok = mbar_wait(acc_done, 0, abort_flag, kSiteBAcc);
-    if (ok) {
+    // Every compute thread gets here; the epilogue runs only if all of them
+    // completed their waits, so the barrier below is reached by all or none.
+    ok = named_barrier_and(1, 256, ok);
+    // A full tile (always in the fixed layout, where rows past N are clipped
+    // by the tensor map) is staged in the K/V shared memory, which the last
+    // MMA has finished reading, and written with TMA stores. A packed tile
+    // that runs past its sequence is written row by row.
+    const bool tma_tile = !PACKED || j * 128 + 128 <= Nk;
+    if (ok && n_steps > 0 && tma_tile) {
+      tc_fence_after();
+      stage_acc_row<D>(tmem + lane_base + (h == 0 ? 256 : 384),
+                       smem + (h == 0 ? C::kVOff : C::kKOff), t, h == 0 ? 1.0f : scale);
+      fence_proxy_async_smem();
+      named_barrier_sync(1, 256);
+      if (threadIdx.x == 0) {
+#pragma unroll
+        for (int a = 0; a < D / 64; ++a) {
+          tma_store_3d(&tm_dv, smem + C::kVOff + a * 16384, a * 64, sp.k0 + j * 128, zkv);
+          tma_store_3d(&tm_dk, smem + C::kKOff + a * 16384, a * 64, sp.k0 + j * 128, zkv);
+        }
+        bulk_commit_group();
+        bulk_wait_read_all();
+      }
+    } else if (ok) {
       const bool valid = key < Nk;
       const long long kv_z = PACKED ? geom.kv_z : static_cast<long long>(Nk) * D;
       const long long kv_row = PACKED ? geom.kv_row : D;
@@ -506,6 +560,7 @@ template <int D, int MODE, int FEAT>
 __global__ void __launch_bounds__(384, 1)
 bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
               const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+              const __grid_constant__ CUtensorMap tm_dq,
               const float* __restrict__ Lws, const float* __restrict__ Dws,
               __nv_bfloat16* __restrict__ dq, int Hq, int group, SeqGeom geom, int Npad,
               float scale_log2, float scale, KeyWindow win, Softcap cap) {
@@ -789,7 +844,27 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
       mbar_arrive(&ds_full[jj & 1]);
     }
     if (ok && n > 0) ok = mbar_wait(acc_done, 0, abort_flag, kSiteBAcc);
-    if (ok) {
+    // As in the dK/dV kernel: all compute threads take part, and a full tile
+    // goes through shared memory (the Q tile, read by no MMA any more) and a
+    // TMA store; each warpgroup stages its own 64-column half.
+    ok = named_barrier_and(1, 256, ok);
+    const bool tma_tile = !PACKED || i * 128 + 128 <= Nq;
+    if (ok && n > 0 && tma_tile) {
+      tc_fence_after();
+      if (h == 0)
+        stage_acc_row<D, 0, D / 64>(tmem + lane_base + 256, smem + C::kQOff, t, scale);
+      else
+        stage_acc_row<D, D / 64, D / 32>(tmem + lane_base + 256, smem + C::kQOff, t, scale);
+      fence_proxy_async_smem();
+      named_barrier_sync(1, 256);
+      if (threadIdx.x == 0) {
+#pragma unroll
+        for (int a = 0; a < D / 64; ++a)
+          tma_store_3d(&tm_dq, smem + C::kQOff + a * 16384, a * 64, sp.q0 + i * 128, zq);
+        bulk_commit_group();
+        bulk_wait_read_all();
+      }
+    } else if (ok) {
       const bool valid = row < Nq;
       const long long o_z = PACKED ? geom.o_z : static_cast<long long>(Nq) * D;
       const long long o_row = PACKED ? geom.o_row : D;

@@ -34,7 +34,8 @@
 // take turns: K0, V0, K1, V1, ... Each 128 x D tile is stored as D/64
 // column blocks of 128 rows x 128 bytes, 128-byte swizzled, exactly as the
 // TMA writes it. That is the canonical K-major SW128 layout for Q and K and
-// the MN-major SW128 layout for V.
+// the MN-major SW128 layout for V. At the end, tile t's bf16 O is staged in
+// Q_t's slot in the same layout and written with a TMA store.
 #pragma once
 
 #include "geometry.cuh"
@@ -79,7 +80,8 @@ static_assert(2 * kFwdRegsSoftmax + kFwdRegsSmall <= 3 * kFwdRegsLaunch, "regist
 template <int D, int MODE, int FEAT>
 __global__ void __launch_bounds__(384, 1)
 fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-           const __grid_constant__ CUtensorMap tm_v, __nv_bfloat16* __restrict__ out,
+           const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
+           __nv_bfloat16* __restrict__ out,
            float* __restrict__ lse_out, int Hq, int group, SeqGeom geom, float scale_log2,
            KeyWindow win, Softcap cap, int one_tile) {
   constexpr bool SOFTCAP = (FEAT & kFeatSoftcap) != 0;
@@ -460,10 +462,52 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
     // Tile 1 of a one-tile CTA holds rows of the next CTA: never write them.
     const bool present = r_first < Nq && (t == 0 || !one_tile);
     if (ok) ok = mbar_wait(&o_full[t], 0, abort_flag, kSiteOFull);
-    if (ok || (present && n == 0)) {
-      const bool has_o = n > 0;
+    const bool write = ok || (present && n == 0);
+    // The warpgroup writes its tile through shared memory and a TMA store when
+    // every thread may write and the tile is whole (the fixed layout clips rows
+    // past Nq through the tensor map). Q_t's slot is free: tile t's last S MMA
+    // finished before o_full[t]. Otherwise each thread stores its own row.
+    const bool all_write = named_barrier_and(1 + t, 128, write);
+    const bool tma_tile = present && (!PACKED || r_first + 128 <= Nq);
+    const bool has_o = n > 0;
+    const float inv_l = (l_mma > 0.f) ? 1.0f / l_mma : 0.f;
+    if (all_write && tma_tile) {
       if (has_o) tc_fence_after();
-      const float inv_l = (l_mma > 0.f) ? 1.0f / l_mma : 0.f;
+      uint8_t* tile = smem + C::kQOff + t * C::kTileBytes;
+      const int tr = quad * 32 + lane;                       // row within the tile
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t o[32];
+        if (has_o) {
+          tmem_ld32(t_o + c * 32, o);
+          tmem_ld_wait(o);
+        } else {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) o[e] = 0u;
+        }
+        uint32_t pk[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e)
+          pk[e] = pack_bf16x2(u2f(o[2 * e]) * inv_l, u2f(o[2 * e + 1]) * inv_l);
+        uint8_t* rowp = tile + (c >> 1) * 16384 + tr * 128;
+#pragma unroll
+        for (int qq = 0; qq < 4; ++qq) {
+          const int ch = (c & 1) * 4 + qq;
+          *reinterpret_cast<uint4*>(rowp + ((ch ^ (tr & 7)) << 4)) =
+              make_uint4(pk[4 * qq], pk[4 * qq + 1], pk[4 * qq + 2], pk[4 * qq + 3]);
+        }
+      }
+      fence_proxy_async_smem();
+      named_barrier_sync(1 + t, 128);
+      if (quad == 0 && lane == 0) {
+#pragma unroll
+        for (int a = 0; a < D / 64; ++a)
+          tma_store_3d(&tm_o, tile + a * 16384, a * 64, sp.q0 + r_first, zq);
+        bulk_commit_group();
+        bulk_wait_read_all();
+      }
+    } else if (write) {
+      if (has_o) tc_fence_after();
       const long long o_z = PACKED ? geom.o_z : static_cast<long long>(Nq) * D;
       const long long o_row = PACKED ? geom.o_row : D;
       __nv_bfloat16* orow = out + zq * o_z + (sp.q0 + (row < Nq ? row : 0)) * o_row;
@@ -479,7 +523,8 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
         }
         uint32_t pk[16];
 #pragma unroll
-        for (int e = 0; e < 16; ++e) pk[e] = pack_bf16x2(u2f(o[2 * e]) * inv_l, u2f(o[2 * e + 1]) * inv_l);
+        for (int e = 0; e < 16; ++e)
+          pk[e] = pack_bf16x2(u2f(o[2 * e]) * inv_l, u2f(o[2 * e + 1]) * inv_l);
         if (row < Nq) {
           uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
           dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
@@ -488,10 +533,10 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
           dst[3] = make_uint4(pk[12], pk[13], pk[14], pk[15]);
         }
       }
-      if (row < Nq)
-        lse_out[zq * (PACKED ? geom.lse_z : static_cast<long long>(Nq)) + sp.q0 + row] =
-            (l_run > 0.f) ? (m_run + __log2f(l_run)) * 0.69314718055994531f : -INFINITY;
     }
+    if (write && row < Nq)
+      lse_out[zq * (PACKED ? geom.lse_z : static_cast<long long>(Nq)) + sp.q0 + row] =
+          (l_run > 0.f) ? (m_run + __log2f(l_run)) * 0.69314718055994531f : -INFINITY;
   }
 
   tc_fence_before();
