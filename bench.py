@@ -282,7 +282,7 @@ def run_reference(args):
             "ms_per_step": cb["seconds"] * 1e3 / max(1, args.steps),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic (seeded iid N(0,1) -> bf16 inputs, upcast to float64)",
-            "config": config_dict(w, args.gpus),
+            "config": dict(config_dict(w, args.gpus), mode="step"),
             "cpu_baseline": {k: cb[k] for k in ("value", "unit", "cores", "kind", "sample")},
             "e2e": {"value": cb["value"], "unit": UNIT, "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
@@ -541,9 +541,10 @@ def run_ours(args):
                for kn, (n, ms) in prof.items()}
 
     # End to end through the public API from pinned host buffers: every step
-    # copies q, k, v, dO in, runs forward + backward, and copies dq, dk, dv
-    # out (forward mode: q, k, v in; o, lse out). Copies in, compute and
-    # copies out run on three streams over two sets of device tensors: step
+    # copies q, k, v, dO in, runs forward + backward, and copies o, lse, dq,
+    # dk and dv out (forward mode: q, k, v in; o, lse out). Copies in,
+    # compute and copies out run on three streams over two sets of device
+    # tensors: step
     # i+1's inputs cross PCIe while step i computes and step i-1's results
     # come back. Events order each set's reuse.
     pin = [t.pin_memory() for t in host]
@@ -553,8 +554,10 @@ def run_ours(args):
     for _ in range(2):
         st = {"in": [torch.empty_like(t) for t in (q, k, v, do)[:n_in]],
               "o": torch.empty_like(o), "lse": torch.empty_like(lse)}
+        # Every output of the step leaves the device: o and lse, and in step
+        # mode dq, dk and dv as well.
         st["out"] = [st["o"], st["lse"]] if fwd_only else \
-            [torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)]
+            [st["o"], st["lse"], torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)]
         sets.append(st)
     host_out = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in sets[0]["out"]]
     s_in, s_comp, s_out = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
@@ -567,7 +570,7 @@ def run_ours(args):
         ea.attn_fwd(qb, kb, vb, st["o"], st["lse"], scale=w.scale, causal=w.causal,
                     stream=s_comp)
         if not fwd_only:
-            dq_b, dk_b, dv_b = st["out"]
+            dq_b, dk_b, dv_b = st["out"][2:]
             ea.attn_bwd(qb, kb, vb, st["o"], st["lse"], st["in"][3], dq_b, dk_b, dv_b, ws,
                         scale=w.scale, causal=w.causal, stream=s_comp)
 
@@ -618,7 +621,7 @@ def run_ours(args):
         del pin, host_out
         torch.cuda.empty_cache()
         extra = []
-        for tw in (workloads.C3_CAUSAL, workloads.C4):
+        for tw in (workloads.C3_CAUSAL, workloads.C3_FULL, workloads.C3_STRESS, workloads.C4):
             r = fwd_target(ea, torch, tw)
             r["frac_of_measured_peak"] = r["tflops"] / peaks["bf16_tflops"]
             extra.append(r)

@@ -155,25 +155,48 @@ def attn_bwd_workspace_size(B, Hq, N, d) -> int:
     return int(load_library().attn_bwd_workspace_size(B, Hq, N, d))
 
 
-def attn_bwd(q, k, v, o, lse, dO, dq=None, dk=None, dv=None, workspace=None, scale=None,
-             causal=False, stream=None):
-    """Backward pass; returns (dq, dk, dv). Allocates outputs/workspace if not given."""
+def _check_bwd_inputs(q, k, v, o, lse, dO):
+    """Shapes and dtypes of the fixed-length backward's inputs. The library
+    builds its tensor maps from q's and k's shapes, so a smaller o, dO or lse
+    would be read past its end: it is refused here, before any launch."""
     import torch
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (o, "o"), (lse, "lse"), (dO, "dO")):
+        if not isinstance(t, torch.Tensor):
+            raise TypeError(f"{n} must be a torch.Tensor")
+    if q.dim() != 4:
+        raise ValueError(f"q must be [B, Hq, N, d], got shape {tuple(q.shape)}")
     B, Hq, N, d = q.shape
-    Hkv = k.shape[1]
+    Hkv = k.shape[1] if k.dim() == 4 else -1
     if k.shape != (B, Hkv, N, d) or v.shape != k.shape or o.shape != q.shape \
             or dO.shape != q.shape or lse.shape != (B, Hq, N):
         raise ValueError("shape mismatch among q, k, v, o, lse, dO")
     for t, n in ((q, "q"), (k, "k"), (v, "v"), (o, "o"), (dO, "dO")):
         _check_dtype(t, torch.bfloat16, n)
     _check_dtype(lse, torch.float32, "lse")
+    return B, Hq, Hkv, N, d
+
+
+def _check_grad_outputs(dq, dk, dv, q, k, v):
+    """The gradient outputs must match q, k, v in shape and be bf16: the
+    kernels store whole tiles into them through tensor maps sized from q/k."""
+    import torch
+    for t, n, ref in ((dq, "dq", q), (dk, "dk", k), (dv, "dv", v)):
+        if not isinstance(t, torch.Tensor):
+            raise TypeError(f"{n} must be a torch.Tensor")
+        _check_dtype(t, torch.bfloat16, n)
+        if t.shape != ref.shape:
+            raise ValueError(f"{n} shape {tuple(t.shape)} does not match {tuple(ref.shape)}")
+
+
+def attn_bwd(q, k, v, o, lse, dO, dq=None, dk=None, dv=None, workspace=None, scale=None,
+             causal=False, stream=None):
+    """Backward pass; returns (dq, dk, dv). Allocates outputs/workspace if not given."""
+    import torch
+    B, Hq, Hkv, N, d = _check_bwd_inputs(q, k, v, o, lse, dO)
     dq = torch.empty_like(q) if dq is None else dq
     dk = torch.empty_like(k) if dk is None else dk
     dv = torch.empty_like(v) if dv is None else dv
-    for t, n, ref in ((dq, "dq", q), (dk, "dk", k), (dv, "dv", v)):
-        _check_dtype(t, torch.bfloat16, n)
-        if t.shape != ref.shape:
-            raise ValueError(f"{n} shape mismatch")
+    _check_grad_outputs(dq, dk, dv, q, k, v)
     need = attn_bwd_workspace_size(B, Hq, N, d)
     if workspace is None:
         workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
@@ -196,9 +219,10 @@ def attn_bwd_noalloc(q, k, v, o, lse, dO, dq, dk, dv, scale=None, causal=False, 
     memory when the backward runs. The scratch is a fixed 8 MiB device array
     inside the library (shapes with B * Hq * ceil128(N) > 1048576 are rejected),
     and the output tensors must be passed in. Calls that
-    overlap on the GPU share that array and race. Returns (dq, dk, dv)."""
-    B, Hq, N, d = q.shape
-    Hkv = k.shape[1]
+    overlap on the GPU share that array and race. Returns (dq, dk, dv).
+    Shapes and dtypes are checked as in attn_bwd before anything is launched."""
+    B, Hq, Hkv, N, d = _check_bwd_inputs(q, k, v, o, lse, dO)
+    _check_grad_outputs(dq, dk, dv, q, k, v)
     scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
     lib = load_library()
     with _device_guard(q, k, v, o, lse, dO, dq, dk, dv):

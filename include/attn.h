@@ -102,7 +102,13 @@ attn_status attn_bwd(const void* q, const void* k, const void* v, const void* o,
                      void* workspace, size_t workspace_bytes, int B, int Hq, int Hkv, int N,
                      int d, float scale, int causal, attn_stream_t stream);
 
-/* Bytes of workspace attn_bwd needs for this shape (0 for an empty problem). */
+/*
+ * Bytes of workspace attn_bwd needs for this shape (0 for an empty problem).
+ * The pages have no counterpart: it exists because this library never
+ * allocates, so the caller sizes and owns the backward's scratch (two fp32
+ * rows per query, padded to a multiple of 128 per head). d is accepted for
+ * symmetry with the other calls and does not change the size.
+ */
 size_t attn_bwd_workspace_size(int B, int Hq, int N, int d);
 
 /*
@@ -214,6 +220,10 @@ attn_status attn_bwd_varlen(const void* q, const void* k, const void* v, const v
                             attn_stream_t stream);
 
 /*
+ * attn_check_status: own design; the pages have no counterpart. The kernels
+ * never trap: a pipeline wait that gives up, or packed offsets that had to be
+ * clipped, is recorded in a device status word instead, and this call turns
+ * that word into a status code and a message.
  * Synchronises `stream`, then reads and clears the device status word.
  * Returns ATTN_ERR_TIMEOUT if a kernel gave up on a wait since the last
  * check, ATTN_ERR_ARG if a varlen call met invalid cu_seqlens offsets,
@@ -232,8 +242,17 @@ attn_status attn_check_status(attn_stream_t stream);
  */
 attn_status attn_selftest_wait_timeout(attn_stream_t stream);
 
-/* Message of the last error on the calling thread ("" if none). The library
- * owns the string. It stays valid until the next call on the same thread. */
+/*
+ * Message of the last error on the calling thread ("" if none). The library
+ * owns the string. It stays valid until the next call on the same thread.
+ * tokenwerk.de "FlashAttention", section "Fehler und Leistungsversprechen
+ * richtig einordnen": when a kernel is missing, the version, the GPU and the
+ * input shape are checked first and the exact message is recorded. Every
+ * non-OK status therefore comes with a message that names the argument, the
+ * shape or the CUDA call that failed (for example "head dim 96 not supported
+ * (built: 64, 128)" or "this library is built for sm_100a (B200); device 0 is
+ * sm_90").
+ */
 const char* attn_get_last_error(void);
 
 /*

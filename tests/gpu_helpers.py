@@ -77,3 +77,40 @@ def sample_rows(N, rng, extra=24):
         rows = sorted(rows[i] for i in keep) + [0, N - 1]
     rows += list(rng.integers(0, N, size=extra))
     return np.array(sorted(set(int(r) for r in rows)))
+
+
+# Relative error of one bf16 round-to-nearest: half a unit in the last place
+# of an 8-bit significand.
+BF16_HALF_ULP_REL = 2.0 ** -9
+# Slack for the kernel's fp32 arithmetic around P: ex2.approx and the softcap's
+# rcp.approx (relative errors near 2^-22), the fp32 tensor-core accumulation,
+# and the fp32 row sums. Far above their sum at these sizes, far below 2^-9.
+FP32_PATH_REL = 2e-4
+
+
+def p_rounding_bound(q, k, v, scale, causal, window=(-1, -1), softcap=0.0):
+    """Element-wise error bound for O when P is rounded to bf16 before the PV
+    product and the output is rounded to bf16 once.
+
+    Derivation (own, from the arithmetic; the pages give the definition only).
+    Let w_j be the exact softmax weights of a row and O = sum_j w_j v_j. The
+    kernel multiplies V by p_j (1 + d_j), |d_j| <= u with u = 2^-9 + fp32
+    slack, and divides by the sum of the same rounded p_j. Then
+        O_kernel - O = sum_j w_j d_j (v_j - O) / (1 + sum_j w_j d_j),
+    so |O_kernel - O| <= u / (1 - u) * sum_j w_j |v_j - O| per output column.
+    Rounding the fp32 result to bf16 adds at most 2^-9 |O_kernel|. Returns the
+    bound with the float64 oracle's weights, shaped like O [B, Hq, Nq, d]."""
+    q64, k64, v64 = (oracle.to_f64(t) for t in (q, k, v))
+    B, Hq, Nq, d = q64.shape
+    G = Hq // k64.shape[1]
+    u = BF16_HALF_ULP_REL + FP32_PATH_REL
+    out = np.empty((B, Hq, Nq, d))
+    for b in range(B):
+        for h in range(Hq):
+            kk, vv = k64[b, h // G], v64[b, h // G]
+            s = oracle.scores(q64[b, h], kk, scale, causal, window=window, softcap=softcap)
+            w, _, _ = oracle.softmax_rows(s)
+            o = w @ vv
+            spread = np.einsum("ij,ijc->ic", w, np.abs(vv[None, :, :] - o[:, None, :]))
+            out[b, h] = u / (1.0 - u) * spread + BF16_HALF_ULP_REL * (np.abs(o) + u * spread)
+    return out

@@ -98,6 +98,32 @@ def test_full_size_sampled_rows(w):
     assert np.all(o_cpu >= vmin[:, :, None, :] - 2e-2)
 
 
+WHOLE_HEAD_WORKLOADS = [workloads.C3_CAUSAL, workloads.C3_FULL, workloads.C3_STRESS, workloads.C4,
+                        workloads.C5]
+
+
+@pytest.mark.parametrize("w", WHOLE_HEAD_WORKLOADS, ids=lambda w: w.name)
+def test_full_size_whole_heads(w):
+    """Every element of whole heads at full size, against the row-chunked
+    oracle (each row of S and P is still materialised over all keys). c3
+    (causal, non-causal, Q x4) and c4 compare two heads, the training-step
+    workload c5 compares the three heads its backward test checks."""
+    q, k, v = workloads.make_inputs(w, with_grad_out=False)
+    o, lse = gpu_fwd(q, k, v, w.scale, w.causal)
+    o_cpu = o.float().cpu().numpy()
+    lse_cpu = lse.cpu().numpy()
+    if w is workloads.C5:
+        heads = [(0, 0), (3, 7), (w.B - 1, w.Hq - 1)]
+    else:
+        heads = [(0, w.Hq // 3), (w.B - 1, w.Hq - 1)]
+    G = w.Hq // w.Hkv
+    for b, h in heads:
+        hk = h // G
+        o_ref, lse_ref = oracle.attention_head(oracle.to_f64(q[b, h]), oracle.to_f64(k[b, hk]),
+                                               oracle.to_f64(v[b, hk]), w.scale, w.causal)
+        assert_fwd_close(o_cpu[b, h], lse_cpu[b, h], o_ref, lse_ref, f"{w.name} head ({b},{h})")
+
+
 def test_repeat_runs_are_bitwise_identical():
     w = workloads.small("det", 2, 4, 2, 700, 128, True, seed=3, backward=False)
     q, k, v = workloads.make_inputs(w, with_grad_out=False)

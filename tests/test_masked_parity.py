@@ -17,7 +17,8 @@ import torch
 import exact_attention_105_b200 as ea
 import oracle
 import workloads
-from tests.gpu_helpers import GRAD_REL_TOL, LSE_TOL, O_TOL, max_err, to_dev
+from tests.gpu_helpers import (GRAD_REL_TOL, LSE_TOL, O_TOL, max_err, p_rounding_bound,
+                               to_dev)
 
 pytestmark = pytest.mark.gpu
 
@@ -249,9 +250,6 @@ SOFTCAP_CASES = [
     (1, 2, 2, 257, 257, 64, True, (-1, -1), 1.0, 4.0),       # nearly uniform weights
     (1, 4, 2, 200, 700, 128, True, (128, -1), 10.0, 2.0),    # window, Nq < Nk, GQA
     (1, 2, 2, 700, 200, 64, True, (-1, -1), 20.0, 2.0),      # rows without keys
-    # At Q x4 this case measured max|O - O_ref| = 1.01e-2: the bf16 rounding of
-    # P near one-hot rows, as in the uncapped Q x4 stress; large-logit capping
-    # is covered by the Q x4 cases above.
     (2, 8, 2, 384, 640, 128, False, (96, 64), 30.0, 2.0),
 ]
 
@@ -268,6 +266,46 @@ def test_softcap_fwd_bwd(case):
     assert_masked_fwd_close(o, lse, o_ref, lse_ref, str(case))
     refs = oracle.attention_backward(q, k, v, do, scale, causal, window=window, softcap=cap)
     assert_masked_grads_close(got, refs, str(case), causal, window)
+
+
+def test_softcap_q4_within_derived_rounding_bound():
+    """Cap 30 at Q x4, window (96, 64), Nq < Nk, GQA. Large logits make many
+    rows nearly one-hot with |O| up to about 3, where the bf16 output rounding
+    alone can reach 7.8e-3 and the bf16 rounding of P adds to it, so the fixed
+    1e-2 bound of the workload configurations is not the right yardstick here.
+    Instead every element must lie within the bound that follows from those
+    two roundings (``p_rounding_bound``), and the maximum error must be at most
+    twice that of a plain bf16 attention on the same inputs (the upstream test
+    rule, hysenlabs.com, section "Tests, BSD-3-Clause und Zitierpraxis").
+    The gradients keep the usual 2e-2 * max|ref| bound."""
+    B, Hq, Hkv, Nq, Nk, d, causal, window, cap, qm = (2, 8, 2, 384, 640, 128, False, (96, 64),
+                                                       30.0, 4.0)
+    q, k, v, do = workloads.make_inputs_qk(B, Hq, Hkv, Nq, Nk, d, seed=Nq + 11 * Nk + d,
+                                           q_mult=qm)
+    scale = d ** -0.5
+    (o, lse), got = run_fwd_bwd(q, k, v, do, scale, causal, window, softcap=cap)
+    o_ref, lse_ref = oracle.attention_forward(q, k, v, scale, causal, window=window, softcap=cap)
+    o_np = o.float().cpu().numpy()
+    assert np.all(np.isfinite(o_np))
+    err = np.abs(o_np - o_ref)
+    bound = p_rounding_bound(q, k, v, scale, causal, window=window, softcap=cap)
+    worst = np.unravel_index(int(np.argmax(err - bound)), err.shape)
+    assert np.all(err <= bound), \
+        f"|O-O_ref| = {err[worst]:.3e} > bound {bound[worst]:.3e} at {worst} (O_ref {o_ref[worst]:.4f})"
+    el, _ = max_err(lse.cpu().numpy(), lse_ref)
+    assert el <= LSE_TOL, el
+    # Plain bf16 attention with the same cap and mask, materialised in torch.
+    qd, kd, vd = to_dev(q, k, v)
+    kd, vd = (t.repeat_interleave(Hq // Hkv, dim=1) for t in (kd, vd))
+    s = torch.matmul(qd, kd.transpose(-1, -2)) * scale
+    s = cap * torch.tanh(s / cap)
+    vis = torch.from_numpy(oracle.visible(np.arange(Nq), Nq, Nk, causal, window)).cuda()
+    s = s.masked_fill(~vis, float("-inf"))
+    naive = torch.matmul(torch.softmax(s, dim=-1).to(torch.bfloat16), vd).float().cpu().numpy()
+    e_naive = float(np.abs(naive - o_ref).max())
+    assert float(err.max()) <= 2.0 * e_naive, (float(err.max()), e_naive)
+    refs = oracle.attention_backward(q, k, v, do, scale, causal, window=window, softcap=cap)
+    assert_masked_grads_close(got, refs, "softcap30_q4", causal, window)
 
 
 def test_softcap_changes_the_result():
