@@ -89,18 +89,60 @@ def _check(status: int):
         raise AttnError(status, msg)
 
 
+class _OnDevice:
+    """Makes CUDA device `index` current for the duration of a call, and
+    exposes its current stream. When the device is already current (the
+    usual case) it changes nothing, which keeps the per-call host cost low."""
+
+    __slots__ = ("index", "prev")
+
+    def __init__(self, index):
+        self.index = index
+        self.prev = None
+
+    def __enter__(self):
+        import torch
+        cur = torch.cuda.current_device()
+        if cur != self.index:
+            self.prev = cur
+            torch.cuda.set_device(self.index)
+        return self
+
+    def __exit__(self, *exc):
+        if self.prev is not None:
+            import torch
+            torch.cuda.set_device(self.prev)
+        return False
+
+    def stream(self, stream):
+        """The handle to launch on: `stream` if given, else the device's current stream."""
+        if stream is not None:
+            return ctypes.c_void_p(stream.cuda_stream)
+        import torch
+        raw = getattr(torch._C, "_cuda_getCurrentRawStream", None)
+        if raw is not None:
+            return ctypes.c_void_p(raw(self.index))
+        return ctypes.c_void_p(torch.cuda.current_stream(self.index).cuda_stream)
+
+
 def _device_guard(*tensors):
     """All tensor arguments must live on one CUDA device. The call then runs
     with that device current (the library launches on the current device)."""
     import torch
-    devs = {t.device for t in tensors if isinstance(t, torch.Tensor)}
-    if len(devs) != 1:
-        raise ValueError(f"all tensors must be on one device, got {sorted(map(str, devs))}")
-    dev = devs.pop()
-    if dev.type != "cuda":
-        raise ValueError(f"tensors must be CUDA tensors (the library takes device pointers), "
-                         f"got {dev}")
-    return torch.cuda.device(dev)
+    idx = None
+    for t in tensors:
+        if not isinstance(t, torch.Tensor):
+            continue
+        i = t.get_device()
+        if idx is None:
+            idx = i
+        elif i != idx:
+            devs = sorted({str(x.device) for x in tensors if isinstance(x, torch.Tensor)})
+            raise ValueError(f"all tensors must be on one device, got {devs}")
+    if idx is None or idx < 0:
+        raise ValueError("tensors must be CUDA tensors (the library takes device pointers), "
+                         f"got {tensors[0].device if tensors else None}")
+    return _OnDevice(idx)
 
 
 def _stream_handle(stream):
@@ -144,10 +186,10 @@ def attn_fwd(q, k, v, o=None, lse=None, scale=None, causal=False, stream=None):
         raise ValueError("o/lse shape mismatch")
     scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
     lib = load_library()
-    with _device_guard(q, k, v, o, lse):
+    with _device_guard(q, k, v, o, lse) as g:
         _check(lib.attn_fwd(_dev_ptr(q, "q"), _dev_ptr(k, "k"), _dev_ptr(v, "v"), _dev_ptr(o, "o"),
                             _dev_ptr(lse, "lse"), B, Hq, Hkv, N, d, scale, int(bool(causal)),
-                            _stream_handle(stream)))
+                            g.stream(stream)))
     return o, lse
 
 
@@ -202,12 +244,12 @@ def attn_bwd(q, k, v, o, lse, dO, dq=None, dk=None, dv=None, workspace=None, sca
         workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
     scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
     lib = load_library()
-    with _device_guard(q, k, v, o, lse, dO, dq, dk, dv, workspace):
+    with _device_guard(q, k, v, o, lse, dO, dq, dk, dv, workspace) as g:
         _check(lib.attn_bwd(_dev_ptr(q, "q"), _dev_ptr(k, "k"), _dev_ptr(v, "v"), _dev_ptr(o, "o"),
                             _dev_ptr(lse, "lse"), _dev_ptr(dO, "dO"), _dev_ptr(dq, "dq"),
                             _dev_ptr(dk, "dk"), _dev_ptr(dv, "dv"), _dev_ptr(workspace, "workspace"),
                             workspace.numel() * workspace.element_size(),
-                            B, Hq, Hkv, N, d, scale, int(bool(causal)), _stream_handle(stream)))
+                            B, Hq, Hkv, N, d, scale, int(bool(causal)), g.stream(stream)))
     return dq, dk, dv
 
 
@@ -225,12 +267,12 @@ def attn_bwd_noalloc(q, k, v, o, lse, dO, dq, dk, dv, scale=None, causal=False, 
     _check_grad_outputs(dq, dk, dv, q, k, v)
     scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
     lib = load_library()
-    with _device_guard(q, k, v, o, lse, dO, dq, dk, dv):
+    with _device_guard(q, k, v, o, lse, dO, dq, dk, dv) as g:
         _check(lib.attn_bwd_noalloc(_dev_ptr(q, "q"), _dev_ptr(k, "k"), _dev_ptr(v, "v"),
                                     _dev_ptr(o, "o"), _dev_ptr(lse, "lse"), _dev_ptr(dO, "dO"),
                                     _dev_ptr(dq, "dq"), _dev_ptr(dk, "dk"), _dev_ptr(dv, "dv"),
                                     B, Hq, Hkv, N, d, scale, int(bool(causal)),
-                                    _stream_handle(stream)))
+                                    g.stream(stream)))
     return dq, dk, dv
 
 
@@ -269,11 +311,11 @@ def attn_fwd_masked(q, k, v, o=None, lse=None, scale=None, causal=False, window=
     scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
     wl, wr = _window(window)
     lib = load_library()
-    with _device_guard(q, k, v, o, lse):
+    with _device_guard(q, k, v, o, lse) as g:
         _check(lib.attn_fwd_masked(_dev_ptr(q, "q"), _dev_ptr(k, "k"), _dev_ptr(v, "v"),
                                    _dev_ptr(o, "o"), _dev_ptr(lse, "lse"), B, Hq, Hkv, Nq, Nk, d,
                                    scale, int(bool(causal)), wl, wr, _softcap(softcap),
-                                   _stream_handle(stream)))
+                                   g.stream(stream)))
     return o, lse
 
 
@@ -302,14 +344,14 @@ def attn_bwd_masked(q, k, v, o, lse, dO, dq=None, dk=None, dv=None, workspace=No
     scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
     wl, wr = _window(window)
     lib = load_library()
-    with _device_guard(q, k, v, o, lse, dO, dq, dk, dv, workspace):
+    with _device_guard(q, k, v, o, lse, dO, dq, dk, dv, workspace) as g:
         _check(lib.attn_bwd_masked(_dev_ptr(q, "q"), _dev_ptr(k, "k"), _dev_ptr(v, "v"),
                                    _dev_ptr(o, "o"), _dev_ptr(lse, "lse"), _dev_ptr(dO, "dO"),
                                    _dev_ptr(dq, "dq"), _dev_ptr(dk, "dk"), _dev_ptr(dv, "dv"),
                                    _dev_ptr(workspace, "workspace"),
                                    workspace.numel() * workspace.element_size(),
                                    B, Hq, Hkv, Nq, Nk, d, scale, int(bool(causal)), wl, wr,
-                                   _softcap(softcap), _stream_handle(stream)))
+                                   _softcap(softcap), g.stream(stream)))
     return dq, dk, dv
 
 
@@ -349,12 +391,12 @@ def attn_fwd_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, max_seqle
     scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
     wl, wr = _window(window)
     lib = load_library()
-    with _device_guard(q, k, v, o, lse, cu_seqlens_q, cu_seqlens_k):
+    with _device_guard(q, k, v, o, lse, cu_seqlens_q, cu_seqlens_k) as g:
         _check(lib.attn_fwd_varlen(_dev_ptr(q, "q"), _dev_ptr(k, "k"), _dev_ptr(v, "v"),
                                    _dev_ptr(o, "o"), _dev_ptr(lse, "lse"), cq, ck, B, Hq, Hkv,
                                    total_q, total_k, int(max_seqlen_q), int(max_seqlen_k), d, scale,
                                    int(bool(causal)), wl, wr, _softcap(softcap),
-                                   _stream_handle(stream)))
+                                   g.stream(stream)))
     return o, lse
 
 
@@ -389,7 +431,7 @@ def attn_bwd_varlen(q, k, v, o, lse, dO, cu_seqlens_q, cu_seqlens_k, max_seqlen_
     scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
     wl, wr = _window(window)
     lib = load_library()
-    with _device_guard(q, k, v, o, lse, dO, dq, dk, dv, workspace, cu_seqlens_q, cu_seqlens_k):
+    with _device_guard(q, k, v, o, lse, dO, dq, dk, dv, workspace, cu_seqlens_q, cu_seqlens_k) as g:
         _check(lib.attn_bwd_varlen(_dev_ptr(q, "q"), _dev_ptr(k, "k"), _dev_ptr(v, "v"),
                                    _dev_ptr(o, "o"), _dev_ptr(lse, "lse"), _dev_ptr(dO, "dO"),
                                    _dev_ptr(dq, "dq"), _dev_ptr(dk, "dk"), _dev_ptr(dv, "dv"), cq, ck,
@@ -397,7 +439,7 @@ def attn_bwd_varlen(q, k, v, o, lse, dO, cu_seqlens_q, cu_seqlens_k, max_seqlen_
                                    workspace.numel() * workspace.element_size(), B, Hq, Hkv, total_q,
                                    total_k, int(max_seqlen_q), int(max_seqlen_k), d, scale,
                                    int(bool(causal)), wl, wr, _softcap(softcap),
-                                   _stream_handle(stream)))
+                                   g.stream(stream)))
     return dq, dk, dv
 
 

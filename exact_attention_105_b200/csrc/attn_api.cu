@@ -195,8 +195,36 @@ cudaError_t prepare_kernel(Kern kern, int smem_bytes, KernelSetup& ks, int* regs
 // row stride d, z stride N*d. Packed [total, H, d]: rows = total, z = H, row
 // stride H*d, z stride d. Rows past `rows` read as zeros, and stores to them
 // are dropped.
+// Recently encoded maps, per calling thread: training and serving loops call
+// with the same tensors again and again, and an encode costs about as much
+// host time as the launch. A map depends only on these arguments (it holds
+// the global address, extents and strides, nothing device-specific).
+struct MapKey {
+  const void* base;
+  long long rows, zdim, row_stride, z_stride;
+  int d;
+  bool operator==(const MapKey& o) const {
+    return base == o.base && rows == o.rows && zdim == o.zdim && row_stride == o.row_stride &&
+           z_stride == o.z_stride && d == o.d;
+  }
+};
+struct MapEntry {
+  MapKey key;
+  CUtensorMap map;
+  bool valid;
+};
+constexpr int kMapCacheSize = 16;
+thread_local MapEntry t_map_cache[kMapCacheSize] = {};
+thread_local int t_map_next = 0;
+
 attn_status make_map(CUtensorMap* map, const void* base, int d, long long rows, long long zdim,
                      long long row_stride, long long z_stride) {
+  const MapKey key{base, rows, zdim, row_stride, z_stride, d};
+  for (int i = 0; i < kMapCacheSize; ++i)
+    if (t_map_cache[i].valid && t_map_cache[i].key == key) {
+      *map = t_map_cache[i].map;
+      return ATTN_OK;
+    }
   cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(rows),
                         static_cast<cuuint64_t>(zdim)};
   cuuint64_t strides[2] = {static_cast<cuuint64_t>(row_stride) * 2,
@@ -208,6 +236,11 @@ attn_status make_map(CUtensorMap* map, const void* base, int d, long long rows, 
                         CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(ATTN_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+  MapEntry& e = t_map_cache[t_map_next];
+  t_map_next = (t_map_next + 1) % kMapCacheSize;
+  e.key = key;
+  e.map = *map;
+  e.valid = true;
   return ATTN_OK;
 }
 
@@ -298,6 +331,23 @@ struct Problem {
   attn::Softcap cap;
 };
 
+// Heads per group of the forward's grid order for unmasked problems:
+// consecutive (batch, query head) indices whose K and V together stay well
+// inside L2 (about 48 MB of the 126 MB), rounded down to whole GQA groups.
+// Masked problems (causal, windows) use one group, to keep the heaviest blocks
+// of every head first. Measured on B200 (c3, N 4096 d 128): unmasked 1076 ->
+// 1137-1155 TFLOP/s with groups; causal within 1 %, and 2-4 % slower at N 2048.
+int fwd_head_group(const Problem& p) {
+  const long long all = static_cast<long long>(p.B) * p.Hq;
+  if (p.mask.mode != attn::kMaskNone) return static_cast<int>(all);
+  const int group = p.Hq / p.Hkv;
+  const double kv_bytes_per_head = 2.0 * p.geom.Nk * p.d * 2.0 / group;
+  const double budget = 48.0 * (1 << 20);
+  long long hg = static_cast<long long>(budget / std::max(kv_bytes_per_head, 1.0));
+  hg = std::max<long long>(group, hg - hg % group);
+  return static_cast<int>(std::min<long long>(hg, all));
+}
+
 template <int D, int MODE, int FEAT>
 attn_status launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                        const CUtensorMap& mo, void* o, float* lse, const Problem& p,
@@ -325,7 +375,7 @@ attn_status launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUten
   ProfScope ps(kProfFwd, stream);
   kern<<<grid, Cfg::kThreads, Cfg::kSmemAlloc, stream>>>(
       mq, mk, mv, mo, static_cast<__nv_bfloat16*>(o), lse, p.Hq, p.Hq / p.Hkv, p.geom, scale_log2,
-      p.mask.win, p.cap, one_tile);
+      p.mask.win, p.cap, one_tile, fwd_head_group(p));
   ps.end();
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "fwd kernel launch");

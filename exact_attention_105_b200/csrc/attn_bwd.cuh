@@ -331,19 +331,21 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       auto stage_addr = [&](int s) { return sbase + C::kStageOff + (s % NS) * C::kStageBytes; };
       // dst(tmem) = A_kmajor(smem tile) * B_kmajor(smem tile)^T, K = D
       auto mma_tile_kk = [&](uint32_t dst, uint32_t a, uint32_t bt) {
+        const SDesc ad = sdesc_sw128_split(a, 16, 1024), bd = sdesc_sw128_split(bt, 16, 1024);
+        mma_ss_w<0>(dst, ad.lo, ad.hi, bd.lo, bd.hi, kIdescSS);
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-          mma_ss(dst, sdesc_sw128(a + off, 16, 1024), sdesc_sw128(bt + off, 16, 1024), kIdescSS,
-                 kk > 0 ? 1u : 0u);
+        for (int kk = 1; kk < D / 16; ++kk) {
+          const uint32_t o = ((kk >> 2) * 16384 + (kk & 3) * 32) >> 4;
+          mma_ss_w<1>(dst, ad.lo + o, ad.hi, bd.lo + o, bd.hi, kIdescSS);
         }
       };
       // acc(tmem) += A(tmem, 128 x 128 bf16, split layout) * B(smem tile, MN-major), K = 128
       auto mma_acc = [&](uint32_t acc, uint32_t a_tmem, uint32_t b, bool accumulate) {
+        const SDesc bd = sdesc_sw128_split(b, 16384, 1024);
+        mma_ts_w<-1>(acc, a_tmem + split_col(0), bd.lo, bd.hi, kIdescAcc, accumulate ? 1u : 0u);
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          mma_ts(acc, a_tmem + split_col(kk), sdesc_sw128(b + kk * 2048, 16384, 1024), kIdescAcc,
-                 (accumulate || kk > 0) ? 1u : 0u);
+        for (int kk = 1; kk < 8; ++kk)
+          mma_ts_w<1>(acc, a_tmem + split_col(kk), bd.lo + kk * 128, bd.hi, kIdescAcc);
       };
       bool ok = n_steps > 0 && mbar_wait(kv_full, 0, abort_flag, kSiteBKV) &&
                 mbar_wait(&ld_full[0], 0, abort_flag, kSiteBLoadFull);
@@ -695,11 +697,12 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
       // dP / dS of step jj live in TMEM columns [128, 256) (even jj) or [384, 512) (odd jj).
       auto dp_col = [&](int jj) { return (jj & 1) ? 384u : 128u; };
       auto mma_tile_kk = [&](uint32_t dst, uint32_t a, uint32_t bt) {
+        const SDesc ad = sdesc_sw128_split(a, 16, 1024), bd = sdesc_sw128_split(bt, 16, 1024);
+        mma_ss_w<0>(dst, ad.lo, ad.hi, bd.lo, bd.hi, kIdescSS);
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-          mma_ss(dst, sdesc_sw128(a + off, 16, 1024), sdesc_sw128(bt + off, 16, 1024), kIdescSS,
-                 kk > 0 ? 1u : 0u);
+        for (int kk = 1; kk < D / 16; ++kk) {
+          const uint32_t o = ((kk >> 2) * 16384 + (kk & 3) * 32) >> 4;
+          mma_ss_w<1>(dst, ad.lo + o, ad.hi, bd.lo + o, bd.hi, kIdescSS);
         }
       };
       bool ok = n > 0 && mbar_wait(qd_full, 0, abort_flag, kSiteBLoadFull) && k_wait(0);
@@ -737,11 +740,12 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
           break;
         }
         tc_fence_after();
-        const uint32_t kb = kslot(jj);
+        const SDesc kbd = sdesc_sw128_split(kslot(jj), 16384, 1024);  // dQ += dS K_j
+        const uint32_t dsc = tmem + dp_col(jj);
+        mma_ts_w<-1>(tmem + 256, dsc + split_col(0), kbd.lo, kbd.hi, kIdescAcc, jj > 0 ? 1u : 0u);
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk)                                // dQ += dS K_j
-          mma_ts(tmem + 256, tmem + dp_col(jj) + split_col(kk),
-                 sdesc_sw128(kb + kk * 2048, 16384, 1024), kIdescAcc, (jj > 0 || kk > 0) ? 1u : 0u);
+        for (int kk = 1; kk < 8; ++kk)
+          mma_ts_w<1>(tmem + 256, dsc + split_col(kk), kbd.lo + kk * 128, kbd.hi, kIdescAcc);
         tc_commit(&k_empty[jj % KS]);
       }
       if (ok) tc_commit(acc_done);

@@ -83,7 +83,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
            const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
            __nv_bfloat16* __restrict__ out,
            float* __restrict__ lse_out, int Hq, int group, SeqGeom geom, float scale_log2,
-           KeyWindow win, Softcap cap, int one_tile) {
+           KeyWindow win, Softcap cap, int one_tile, int hg) {
   constexpr bool SOFTCAP = (FEAT & kFeatSoftcap) != 0;
   constexpr bool PACKED = (FEAT & kFeatPacked) != 0;
   static_assert(FEAT == 0 || MODE == kMaskGeneral, "features run in the general mode");
@@ -106,18 +106,29 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
 
   const int warp = warp_id();
   const int lane = lane_id();
-  // 1-D grid, (batch, query head) fastest, then 256-row query block from the
-  // last (heaviest when causal) to the first: every head's heaviest block is
-  // dispatched before any lighter one, which keeps the causal tail short.
+  // 1-D grid over (batch * query head, 256-row query block). The heads are
+  // taken in groups of hg (all of them when hg covers every head); within a
+  // group, (batch, query head) runs fastest and the blocks go from the last
+  // (heaviest when causal) to the first. Causal problems use one group, so
+  // every head's heaviest block is dispatched before any lighter one, which
+  // keeps the tail short. Unmasked problems, whose blocks all cost the same,
+  // use groups whose K and V fit in L2, so a group's blocks reread K/V from
+  // L2 rather than DRAM.
   // Rows per CTA: two 128-row tiles, or one when the problem is too small to
   // fill the GPU with two-tile CTAs (more CTAs, one tile each).
   const int rb = one_tile ? 128 : 256;
   const int nmb = (geom.Nq + rb - 1) / rb;
   const int BH = gridDim.x / nmb;
-  const int bh = blockIdx.x % BH;                  // b * Hq + hq
+  const int per_group = hg * nmb;
+  const int grp = blockIdx.x / per_group;
+  const int g0 = grp * hg;
+  const int gs = min(hg, BH - g0);
+  const int rr = blockIdx.x - grp * per_group;
+  const int mbi = rr / gs;
+  const int bh = g0 + (rr - mbi * gs);             // b * Hq + hq
   const int b = bh / Hq;
   const int hq = bh - b * Hq;
-  const int mb = nmb - 1 - static_cast<int>(blockIdx.x / BH);
+  const int mb = nmb - 1 - mbi;
   const SeqSpan sp = seq_span<PACKED>(geom, b);
   const int Nq = sp.nq, Nk = sp.nk;
   const int m0 = mb * rb;                          // first query row of this CTA
@@ -217,21 +228,21 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
       constexpr uint32_t kIdescQK = idesc_bf16_f32(128, 128, 0, 0);
       constexpr uint32_t kIdescPV = idesc_bf16_f32(128, D, 0, 1);
       auto issue_qk = [&](int t, uint32_t slot) {
-        const uint32_t qa = sbase + C::kQOff + t * C::kTileBytes;
-        const uint32_t ka = sbase + C::kKVOff + slot * C::kTileBytes;
+        const SDesc qd = sdesc_sw128_split(sbase + C::kQOff + t * C::kTileBytes, 16, 1024);
+        const SDesc kd = sdesc_sw128_split(sbase + C::kKVOff + slot * C::kTileBytes, 16, 1024);
+        mma_ss_w<0>(tmem + t * 128, qd.lo, qd.hi, kd.lo, kd.hi, kIdescQK);
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-          mma_ss(tmem + t * 128, sdesc_sw128(qa + off, 16, 1024), sdesc_sw128(ka + off, 16, 1024),
-                 kIdescQK, kk > 0 ? 1u : 0u);
+        for (int kk = 1; kk < D / 16; ++kk) {
+          const uint32_t o = ((kk >> 2) * 16384 + (kk & 3) * 32) >> 4;
+          mma_ss_w<1>(tmem + t * 128, qd.lo + o, qd.hi, kd.lo + o, kd.hi, kIdescQK);
         }
       };
       auto issue_pv = [&](int t, uint32_t slot, bool acc) {
-        const uint32_t va = sbase + C::kKVOff + slot * C::kTileBytes;
+        const SDesc vd = sdesc_sw128_split(sbase + C::kKVOff + slot * C::kTileBytes, 16384, 1024);
+        const uint32_t pa = tmem + t * 128 + 64, od = tmem + 256 + t * 128;
+        mma_ts_w<-1>(od, pa, vd.lo, vd.hi, kIdescPV, acc ? 1u : 0u);
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          mma_ts(tmem + 256 + t * 128, tmem + t * 128 + 64 + kk * 8,
-                 sdesc_sw128(va + kk * 2048, 16384, 1024), kIdescPV, (acc || kk > 0) ? 1u : 0u);
+        for (int kk = 1; kk < 8; ++kk) mma_ts_w<1>(od, pa + kk * 8, vd.lo + kk * 128, vd.hi, kIdescPV);
       };
       auto kv_wait = [&](uint32_t idx) {
         return mbar_wait(&kv_full[idx % NS], (idx / NS) & 1u, abort_flag, kSiteKVFull);

@@ -238,6 +238,34 @@ __device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_
       : "memory");
 }
 
+// MMA forms taking split descriptors. ACC is the accumulate flag when it is
+// known at compile time (every K step after the first); acc_rt is used when
+// ACC is -1.
+template <int ACC>
+__device__ __forceinline__ void mma_ss_w(uint32_t d_tmem, uint32_t a_lo, uint32_t a_hi,
+                                         uint32_t b_lo, uint32_t b_hi, uint32_t idesc,
+                                         uint32_t acc_rt = 0) {
+  const uint32_t acc = ACC < 0 ? acc_rt : static_cast<uint32_t>(ACC);
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t.reg .b64 da, db;\n\t"
+      "setp.ne.b32 p, %6, 0;\n\t"
+      "mov.b64 da, {%1, %2};\n\tmov.b64 db, {%3, %4};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], da, db, %5, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_lo), "r"(a_hi), "r"(b_lo), "r"(b_hi), "r"(idesc), "r"(acc)
+      : "memory");
+}
+template <int ACC>
+__device__ __forceinline__ void mma_ts_w(uint32_t d_tmem, uint32_t a_tmem, uint32_t b_lo,
+                                         uint32_t b_hi, uint32_t idesc, uint32_t acc_rt = 0) {
+  const uint32_t acc = ACC < 0 ? acc_rt : static_cast<uint32_t>(ACC);
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t.reg .b64 db;\n\t"
+      "setp.ne.b32 p, %5, 0;\n\t"
+      "mov.b64 db, {%2, %3};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], db, %4, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "r"(b_lo), "r"(b_hi), "r"(idesc), "r"(acc)
+      : "memory");
+}
 // Shared-memory matrix descriptor for a 128-byte-swizzled operand tile.
 //   start address, leading-dimension byte offset and stride-dimension byte
 //   offset are stored >> 4 in 14-bit fields; bits 46..47 hold the descriptor
@@ -252,6 +280,24 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo_byt
   d |= static_cast<uint64_t>((sbo_bytes >> 4) & 0x3FFFu) << 32;
   d |= static_cast<uint64_t>(1u) << 46;
   d |= static_cast<uint64_t>(2u) << 61;
+  return d;
+}
+
+// The same descriptor as two 32-bit words. The start-address field is the
+// low 14 bits of the low word, and shared-memory offsets stay below 256 KB, so
+// the descriptor of (start + off) is the low word plus off >> 4 with the high
+// word unchanged. An MMA issuer builds a tile's two words once and then pays
+// one 32-bit add per K step: the issuing thread, alone on its warp and
+// sharing an issue slot with the softmax warps, is otherwise the slowest link
+// of the tile loop.
+struct SDesc {
+  uint32_t lo, hi;
+};
+__device__ __forceinline__ SDesc sdesc_sw128_split(uint32_t saddr, uint32_t lbo_bytes,
+                                                   uint32_t sbo_bytes) {
+  SDesc d;
+  d.lo = ((saddr >> 4) & 0x3FFFu) | (((lbo_bytes >> 4) & 0x3FFFu) << 16);
+  d.hi = ((sbo_bytes >> 4) & 0x3FFFu) | (1u << 14) | (2u << 29);
   return d;
 }
 

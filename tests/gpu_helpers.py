@@ -79,12 +79,13 @@ def sample_rows(N, rng, extra=24):
     return np.array(sorted(set(int(r) for r in rows)))
 
 
-# Relative error of one bf16 round-to-nearest: half a unit in the last place
-# of an 8-bit significand.
-BF16_HALF_ULP_REL = 2.0 ** -9
+# Relative error of one bf16 round-to-nearest: the unit roundoff 2^-p of a
+# p = 8 bit significand (7 stored bits and the implicit one). It is reached
+# just above a power of two: 2.0078 rounds to 2.0, an error of 2^-8 * 2.0078.
+BF16_HALF_ULP_REL = 2.0 ** -8
 # Slack for the kernel's fp32 arithmetic around P: ex2.approx and the softcap's
 # rcp.approx (relative errors near 2^-22), the fp32 tensor-core accumulation,
-# and the fp32 row sums. Far above their sum at these sizes, far below 2^-9.
+# and the fp32 row sums. Far above their sum at these sizes, far below 2^-8.
 FP32_PATH_REL = 2e-4
 
 
@@ -94,11 +95,11 @@ def p_rounding_bound(q, k, v, scale, causal, window=(-1, -1), softcap=0.0):
 
     Derivation (own, from the arithmetic; the pages give the definition only).
     Let w_j be the exact softmax weights of a row and O = sum_j w_j v_j. The
-    kernel multiplies V by p_j (1 + d_j), |d_j| <= u with u = 2^-9 + fp32
+    kernel multiplies V by p_j (1 + d_j), |d_j| <= u with u = 2^-8 + fp32
     slack, and divides by the sum of the same rounded p_j. Then
         O_kernel - O = sum_j w_j d_j (v_j - O) / (1 + sum_j w_j d_j),
     so |O_kernel - O| <= u / (1 - u) * sum_j w_j |v_j - O| per output column.
-    Rounding the fp32 result to bf16 adds at most 2^-9 |O_kernel|. Returns the
+    Rounding the fp32 result to bf16 adds at most 2^-8 |O_kernel|. Returns the
     bound with the float64 oracle's weights, shaped like O [B, Hq, Nq, d]."""
     q64, k64, v64 = (oracle.to_f64(t) for t in (q, k, v))
     B, Hq, Nq, d = q64.shape
