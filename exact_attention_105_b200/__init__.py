@@ -117,12 +117,23 @@ class _OnDevice:
     def stream(self, stream):
         """The handle to launch on: `stream` if given, else the device's current stream."""
         if stream is not None:
-            return ctypes.c_void_p(stream.cuda_stream)
+            return stream.cuda_stream
+        return _raw_stream()(self.index)
+
+
+_RAW_STREAM = None
+
+
+def _raw_stream():
+    """A function from a device index to the raw handle of its current stream.
+    torch's C-level accessor costs a fraction of building a Stream object."""
+    global _RAW_STREAM
+    if _RAW_STREAM is None:
         import torch
-        raw = getattr(torch._C, "_cuda_getCurrentRawStream", None)
-        if raw is not None:
-            return ctypes.c_void_p(raw(self.index))
-        return ctypes.c_void_p(torch.cuda.current_stream(self.index).cuda_stream)
+        fn = getattr(torch._C, "_cuda_getCurrentRawStream", None)
+        _RAW_STREAM = fn if fn is not None else \
+            (lambda i: torch.cuda.current_stream(i).cuda_stream)
+    return _RAW_STREAM
 
 
 def _device_guard(*tensors):
@@ -132,7 +143,7 @@ def _device_guard(*tensors):
     idx = None
     for t in tensors:
         if not isinstance(t, torch.Tensor):
-            continue
+            raise TypeError(f"expected torch.Tensor arguments, got {type(t).__name__}")
         i = t.get_device()
         if idx is None:
             idx = i
@@ -152,14 +163,12 @@ def _stream_handle(stream):
 
 
 def _dev_ptr(t, name):
-    import torch
-    if not isinstance(t, torch.Tensor):
-        raise TypeError(f"{name} must be a torch.Tensor")
-    if not t.is_cuda:
-        raise ValueError(f"{name} must be a CUDA tensor (the library takes device pointers)")
+    """The data pointer of a contiguous tensor, as an int (ctypes passes it as
+    void*). Callers run this inside _device_guard, which has already checked
+    that every tensor is a CUDA tensor on one device."""
     if not t.is_contiguous():
         raise ValueError(f"{name} must be contiguous")
-    return ctypes.c_void_p(t.data_ptr())
+    return t.data_ptr()
 
 
 def _check_dtype(t, dtype, name):
@@ -172,20 +181,24 @@ def attn_fwd(q, k, v, o=None, lse=None, scale=None, causal=False, stream=None):
     import torch
     B, Hq, N, d = q.shape
     Hkv = k.shape[1]
-    if k.shape != (B, Hkv, N, d) or v.shape != k.shape:
+    kshape = (B, Hkv, N, d)
+    if k.shape != kshape or v.shape != kshape:
         raise ValueError(f"k/v shape {tuple(k.shape)}/{tuple(v.shape)} does not match q {tuple(q.shape)}")
-    for t, n in ((q, "q"), (k, "k"), (v, "v")):
-        _check_dtype(t, torch.bfloat16, n)
+    bf16 = torch.bfloat16
+    if q.dtype != bf16 or k.dtype != bf16 or v.dtype != bf16:
+        for t, n in ((q, "q"), (k, "k"), (v, "v")):
+            _check_dtype(t, bf16, n)
     if o is None:
         o = torch.empty_like(q)
     if lse is None:
         lse = torch.empty((B, Hq, N), dtype=torch.float32, device=q.device)
-    _check_dtype(o, torch.bfloat16, "o")
-    _check_dtype(lse, torch.float32, "lse")
+    if o.dtype != bf16 or lse.dtype != torch.float32:
+        _check_dtype(o, bf16, "o")
+        _check_dtype(lse, torch.float32, "lse")
     if o.shape != q.shape or lse.shape != (B, Hq, N):
         raise ValueError("o/lse shape mismatch")
     scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
-    lib = load_library()
+    lib = _lib if _lib is not None else load_library()
     with _device_guard(q, k, v, o, lse) as g:
         _check(lib.attn_fwd(_dev_ptr(q, "q"), _dev_ptr(k, "k"), _dev_ptr(v, "v"), _dev_ptr(o, "o"),
                             _dev_ptr(lse, "lse"), B, Hq, Hkv, N, d, scale, int(bool(causal)),

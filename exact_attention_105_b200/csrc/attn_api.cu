@@ -363,19 +363,24 @@ attn_status launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUten
   if (launch_regs != attn::kFwdRegsLaunch)
     return fail(ATTN_ERR_CUDA, "fwd kernel built with %d registers/thread, expected %d",
                 launch_regs, attn::kFwdRegsLaunch);
-  // Two 128-row tiles per CTA share each K/V tile; when that leaves SMs idle,
-  // one tile per CTA doubles the CTAs.
+  // Work items are 256-row query blocks: two 128-row tiles share each K/V
+  // tile. When there are fewer blocks than SMs, 128-row blocks (one tile)
+  // double their number. The grid is persistent: one CTA per SM, or one per
+  // block when there are fewer blocks.
+  attn::FwdSched sched;
+  sched.BH = p.B * p.Hq;
   const long long pairs = static_cast<long long>(p.B) * p.Hq * ((p.geom.Nq + 255) / 256);
-  const int one_tile = pairs < sm_count() ? 1 : 0;
-  const long long blocks = one_tile ? static_cast<long long>(p.B) * p.Hq * ((p.geom.Nq + 127) / 128)
-                                    : pairs;
-  if (blocks > 0x7FFFFFFFLL) return fail(ATTN_ERR_ARG, "problem too large for one launch");
-  dim3 grid(static_cast<unsigned>(blocks));
+  sched.one_tile = pairs < sm_count() ? 1 : 0;
+  sched.nmb = sched.one_tile ? (p.geom.Nq + 127) / 128 : (p.geom.Nq + 255) / 256;
+  sched.hg = fwd_head_group(p);
+  sched.total = static_cast<long long>(sched.BH) * sched.nmb;
+  if (sched.total > 0x7FFFFFFFLL) return fail(ATTN_ERR_ARG, "problem too large for one launch");
+  dim3 grid(static_cast<unsigned>(std::min<long long>(sched.total, sm_count())));
   const float scale_log2 = p.scale * 1.4426950408889634f;
   ProfScope ps(kProfFwd, stream);
   kern<<<grid, Cfg::kThreads, Cfg::kSmemAlloc, stream>>>(
       mq, mk, mv, mo, static_cast<__nv_bfloat16*>(o), lse, p.Hq, p.Hq / p.Hkv, p.geom, scale_log2,
-      p.mask.win, p.cap, one_tile, fwd_head_group(p));
+      p.mask.win, p.cap, sched);
   ps.end();
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "fwd kernel launch");
