@@ -101,9 +101,9 @@ class _OnDevice:
         self.prev = None
 
     def __enter__(self):
-        import torch
-        cur = torch.cuda.current_device()
+        cur = _current_device()
         if cur != self.index:
+            import torch
             self.prev = cur
             torch.cuda.set_device(self.index)
         return self
@@ -122,6 +122,20 @@ class _OnDevice:
 
 
 _RAW_STREAM = None
+_GET_DEVICE = None
+
+
+def _current_device():
+    """The current CUDA device index. After the first call (which goes through
+    torch.cuda.current_device() and so initialises CUDA) it uses torch's C-level
+    getter, skipping the Python-side initialisation checks on every call."""
+    global _GET_DEVICE
+    if _GET_DEVICE is None:
+        import torch
+        idx = torch.cuda.current_device()
+        _GET_DEVICE = getattr(torch._C, "_cuda_getDevice", None) or torch.cuda.current_device
+        return idx
+    return _GET_DEVICE()
 
 
 def _raw_stream():

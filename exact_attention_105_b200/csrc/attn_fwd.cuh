@@ -615,16 +615,24 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
         const float inv_l = (l_mma > 0.f) ? 1.0f / l_mma : 0.f;
         if (has_o) tc_fence_after();
         uint8_t* tile = smem + C::kQOff + (2 * set + t) * C::kTileBytes;
+        // All of the row's O columns are loaded before one wait (the S and P
+        // registers are dead here), so the loads overlap.
+        uint32_t oall[D / 32][32];
+        if (has_o) {
+#pragma unroll
+          for (int c = 0; c < D / 32; ++c) tmem_ld32(t_o + c * 32, oall[c]);
+          tmem_ld_wait(oall[0]);
+#pragma unroll
+          for (int c = 1; c < D / 32; ++c) reg_fence(oall[c]);
+        } else {
+#pragma unroll
+          for (int c = 0; c < D / 32; ++c)
+#pragma unroll
+            for (int e = 0; e < 32; ++e) oall[c][e] = 0u;
+        }
 #pragma unroll
         for (int c = 0; c < D / 32; ++c) {
-          uint32_t o[32];
-          if (has_o) {
-            tmem_ld32(t_o + c * 32, o);
-            tmem_ld_wait(o);
-          } else {
-#pragma unroll
-            for (int e = 0; e < 32; ++e) o[e] = 0u;
-          }
+          const uint32_t (&o)[32] = oall[c];
           uint32_t pk[16];
 #pragma unroll
           for (int e = 0; e < 16; ++e)
