@@ -61,9 +61,9 @@ struct FwdCfg {
   static constexpr int kQOff = 0;                         // Q set s, tile t: (2 s + t) tiles in
   static constexpr int kKVOff = 4 * kTileBytes;
   static constexpr int kBarOff = kKVOff + kStages * kTileBytes;
-  // q_full[2] q_empty[2] kv_full[S] kv_empty[S] s_full[2] p_full[2] o_full[2]
-  // o_empty[2] stage_full[4] mma_done[1]
-  static constexpr int kNumBars = 2 + 2 + 2 * kStages + 2 + 2 + 2 + 2 + 4 + 1;
+  // q_full[2] q_empty[2] kv_full[S] kv_empty[S] s_full[2] p_full[2] p_half[2]
+  // o_full[2] o_empty[2] stage_full[4] mma_done[1]
+  static constexpr int kNumBars = 2 + 2 + 2 * kStages + 2 + 2 + 2 + 2 + 2 + 4 + 1;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
   static constexpr int kBytes = kMiscOff + 16;
   static constexpr int kSmemAlloc = kBytes + 1024;         // slack for 1024-B alignment
@@ -75,7 +75,7 @@ struct FwdCfg {
 // Wait-site ids reported in the status word when a wait times out.
 enum FwdSite : int {
   kSiteQFull = 1, kSiteKVFull = 2, kSiteKVEmpty = 3, kSiteSFull = 4, kSitePFull = 5,
-  kSiteOFull = 6, kSiteQEmpty = 7, kSiteOEmpty = 8, kSiteStage = 9
+  kSiteOFull = 6, kSiteQEmpty = 7, kSiteOEmpty = 8, kSiteStage = 9, kSitePHalf = 10
 };
 
 // Register split: launched at kFwdRegsLaunch per thread (384 threads fill the
@@ -179,8 +179,9 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
   uint64_t* kv_full = q_empty + 2;
   uint64_t* kv_empty = kv_full + NS;
   uint64_t* s_full = kv_empty + NS;       // per tile
-  uint64_t* p_full = s_full + 2;          // per tile
-  uint64_t* o_full = p_full + 2;          // per tile: the block's last PV is done
+  uint64_t* p_full = s_full + 2;          // per tile: all of P is in TMEM
+  uint64_t* p_half = p_full + 2;          // per tile: P of keys 0..63 is in TMEM
+  uint64_t* o_full = p_half + 2;          // per tile: the block's last PV is done
   uint64_t* o_empty = o_full + 2;         // per tile: the epilogue has read O
   uint64_t* stage_full = o_empty + 2;     // per (Q set, tile): O staged or written directly
   uint64_t* mma_done = stage_full + 4;
@@ -196,6 +197,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
       mbar_init(&q_empty[i], 1);
       mbar_init(&s_full[i], 1);
       mbar_init(&p_full[i], 128);
+      mbar_init(&p_half[i], 128);
       mbar_init(&o_full[i], 1);
       mbar_init(&o_empty[i], 1);
     }
@@ -283,12 +285,15 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
           mma_ss_w<1>(tmem + t * 128, qd.lo + o, qd.hi, kd.lo + o, kd.hi, kIdescQK);
         }
       };
-      auto issue_pv = [&](int t, uint32_t slot, bool acc) {
+      // O_t += P (keys [64 h, 64 h + 64)) V. P is packed bf16 in TMEM columns
+      // [64, 128) of the tile's S region, 32 columns per half.
+      auto issue_pv_half = [&](int t, uint32_t slot, int h, bool acc) {
         const SDesc vd = sdesc_sw128_split(sbase + C::kKVOff + slot * C::kTileBytes, 16384, 1024);
-        const uint32_t pa = tmem + t * 128 + 64, od = tmem + 256 + t * 128;
-        mma_ts_w<-1>(od, pa, vd.lo, vd.hi, kIdescPV, acc ? 1u : 0u);
+        const uint32_t pa = tmem + t * 128 + 64 + 32 * h, od = tmem + 256 + t * 128;
+        mma_ts_w<-1>(od, pa, vd.lo + 4 * h * 128, vd.hi, kIdescPV, acc ? 1u : 0u);
 #pragma unroll
-        for (int kk = 1; kk < 8; ++kk) mma_ts_w<1>(od, pa + kk * 8, vd.lo + kk * 128, vd.hi, kIdescPV);
+        for (int kk = 1; kk < 4; ++kk)
+          mma_ts_w<1>(od, pa + kk * 8, vd.lo + (4 * h + kk) * 128, vd.hi, kIdescPV);
       };
       auto kv_wait = [&](uint32_t idx) {
         return mbar_wait(&kv_full[idx % NS], (idx / NS) & 1u, abort_flag, kSiteKVFull);
@@ -342,8 +347,10 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
             if (j >= lo && j <= hi) {
               uint32_t& pc = tt ? pc1 : pc0;
               int& oc = tt ? oc1 : oc0;
-              if (!mbar_wait(&p_full[tt], pc & 1u, abort_flag, kSitePFull)) { ok = false; break; }
-              ++pc;
+              // P arrives in two halves: the first half's PV runs while the
+              // softmax still computes the second half. The next S tile
+              // overwrites P, so it follows the second half's PV.
+              if (!mbar_wait(&p_half[tt], pc & 1u, abort_flag, kSitePHalf)) { ok = false; break; }
               // The first accumulation of a block overwrites O_t: the previous
               // block's epilogue must have read it.
               if (j == lo && oc > 0 &&
@@ -352,7 +359,11 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
                 break;
               }
               tc_fence_after();
-              issue_pv(tt, iv % NS, j > lo);
+              issue_pv_half(tt, iv % NS, 0, j > lo);
+              if (!mbar_wait(&p_full[tt], pc & 1u, abort_flag, kSitePFull)) { ok = false; break; }
+              ++pc;
+              tc_fence_after();
+              issue_pv_half(tt, iv % NS, 1, true);
               if (j == hi) {
                 tc_commit(&o_full[tt]);
                 ++oc;
@@ -423,7 +434,6 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
     const int quad = warp & 3;
     const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
     const uint32_t t_s = tmem + lane_base + t * 128;
-    const uint32_t t_p = t_s + 64;
     const uint32_t t_o = tmem + lane_base + 256 + t * 128;
     const int tr = quad * 32 + lane;                       // row within the tile
     uint32_t sc = 0;          // S hand-overs consumed by this tile
@@ -556,12 +566,13 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
         const float2 nm2 = make_float2(neg_m, neg_m);
         float2 ex0 = make_float2(0.f, 0.f), ex1 = make_float2(0.f, 0.f);
         float q0 = 0.f, q1 = 0.f, q2 = 0.f, q3 = 0.f;
-        // All 128 scores are exponentiated into 64 packed bf16 pairs first and
-        // stored with two 32-column TMEM stores at the end: a store after every
-        // 32 columns made each chunk wait for its last exponential before the
-        // next chunk started (measured 4 % slower on 16K-key rows). The S
-        // registers die as the P words are produced, so the peak stays near 150
-        // registers. Two row sums are kept. The exact one (unrounded p, paired
+        // The 128 scores become 64 packed bf16 pairs in registers, stored to
+        // TMEM as two 32-column halves. The first half's store is waited for
+        // only after the third chunk's exponentials, so its latency hides
+        // behind them; a wait right after each 32-column chunk stalled every
+        // chunk (measured 4 % slower on 16K-key rows). The S registers die as
+        // the P words are produced, so the peak stays near 150 registers. Two
+        // row sums are kept. The exact one (unrounded p, paired
         // fp32 adds) gives lse. The other adds the bf16-rounded p that the PV MMA
         // consumes, and O is divided by it, so O's weights sum to one as they do
         // in the definition (a one-hot row returns V exactly).
@@ -584,12 +595,17 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
             pw[e] = pk;
           }
         };
+        // P of keys 0..63 goes to TMEM columns 64..95 of the S region and is
+        // handed over first; keys 64..127 go to columns 96..127.
         emit(r0, 0);
         emit(r1, 16);
+        tmem_st32(t_s + 64, *reinterpret_cast<const uint32_t(*)[32]>(pall));
         emit(r2, 32);
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(&p_half[t]);
         emit(r3, 48);
-        tmem_st32(t_p, *reinterpret_cast<const uint32_t(*)[32]>(pall));
-        tmem_st32(t_p + 32, *reinterpret_cast<const uint32_t(*)[32]>(pall + 32));
+        tmem_st32(t_s + 96, *reinterpret_cast<const uint32_t(*)[32]>(pall + 32));
         const float2 ex = fadd2(ex0, ex1);
         l_run += ex.x + ex.y;
         l_mma += (q0 + q1) + (q2 + q3);
