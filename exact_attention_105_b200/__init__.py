@@ -280,12 +280,12 @@ def attn_bwd(q, k, v, o, lse, dO, dq=None, dk=None, dv=None, workspace=None, sca
     return dq, dk, dv
 
 
-NOALLOC_SCRATCH_BYTES = 8 << 20
+NOALLOC_SCRATCH_BYTES = (8 << 20) + 64
 
 
 def attn_bwd_noalloc(q, k, v, o, lse, dO, dq, dk, dv, scale=None, causal=False, stream=None):
     """attn_bwd without a workspace, for callers that must not allocate device
-    memory when the backward runs. The scratch is a fixed 8 MiB device array
+    memory when the backward runs. The scratch is a fixed 8 MiB + 64 byte device array
     inside the library (shapes with B * Hq * ceil128(N) > 1048576 are rejected),
     and the output tensors must be passed in. Calls that
     overlap on the GPU share that array and race. Returns (dq, dk, dv).

@@ -394,6 +394,7 @@ struct BwdArgs {
   const void* dO;
   void *dq, *dk, *dv;
   float *L, *Dv;
+  int* sched;   // the persistent kernels' work counters (zeroed by the preprocess kernel)
 };
 
 template <int D, int MODE, int FEAT>
@@ -404,6 +405,7 @@ attn_status launch_bwd(const BwdArgs& a, const Problem& p, cudaStream_t stream) 
   const float scale_log2 = p.scale * kLog2e;
 
   const long long rows = static_cast<long long>(p.B) * p.Hq * Npad;
+  // dK/dV work items: (batch, KV head, 128-key block); the grid is persistent.
   const long long g1 = static_cast<long long>(pad128(p.geom.Nk) / 128) * p.B * p.Hkv;
   const long long g2 = static_cast<long long>(Npad / 128) * p.B * p.Hq;
   if (rows / 32 > 0x7FFFFFFFLL || g1 > 0x7FFFFFFFLL || g2 > 0x7FFFFFFFLL)
@@ -411,7 +413,7 @@ attn_status launch_bwd(const BwdArgs& a, const Problem& p, cudaStream_t stream) 
   ProfScope p0(kProfBwdPre, stream);
   bwd_pre_kernel<D><<<static_cast<unsigned>(rows / 32), 256, 0, stream>>>(
       static_cast<const __nv_bfloat16*>(a.o), static_cast<const __nv_bfloat16*>(a.dO), a.lse,
-      a.L, a.Dv, p.Hq, p.geom, Npad);
+      a.L, a.Dv, p.Hq, p.geom, Npad, a.sched);
   p0.end();
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "bwd preprocess launch");
@@ -425,16 +427,28 @@ attn_status launch_bwd(const BwdArgs& a, const Problem& p, cudaStream_t stream) 
     return cuda_fail(e, "cudaFuncSetAttribute(dq)");
 
   ProfScope p1(kProfBwdDkdv, stream);
-  k1<<<dim3(static_cast<unsigned>(g1)), DkdvCfg<D>::kThreads, DkdvCfg<D>::kSmemAlloc, stream>>>(
+  const unsigned grid1 = static_cast<unsigned>(std::min<long long>(g1, sm_count()));
+  // Heads numbered key-block-major at the end of the item list: enough for
+  // two items per CTA, so the lightest blocks of those heads come last.
+  const int nkv1 = pad128(p.geom.Nk) / 128;
+  const int tail1 = static_cast<int>(std::min<long long>(static_cast<long long>(p.B) * p.Hkv,
+                                                         (2LL * grid1 + nkv1 - 1) / nkv1));
+  k1<<<dim3(grid1), DkdvCfg<D>::kThreads, DkdvCfg<D>::kSmemAlloc, stream>>>(
       a.mq, a.mk, a.mv, a.mdo, a.mdk, a.mdv, a.L, a.Dv, static_cast<__nv_bfloat16*>(a.dk),
       static_cast<__nv_bfloat16*>(a.dv), p.Hq, group, p.geom, Npad, scale_log2, p.scale,
-      p.mask.win, p.cap);
+      p.mask.win, p.cap, a.sched, static_cast<int>(g1), tail1);
   p1.end();
   if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "bwd dK/dV launch");
   ProfScope p2(kProfBwdDq, stream);
-  k2<<<dim3(static_cast<unsigned>(g2)), DqCfg<D>::kThreads, DqCfg<D>::kSmemAlloc, stream>>>(
+  // dQ work items: (batch, query head, 128-query block); persistent as above.
+  const unsigned grid2 = static_cast<unsigned>(std::min<long long>(g2, sm_count()));
+  const int nqb2 = Npad / 128;
+  const int tail2 = static_cast<int>(std::min<long long>(static_cast<long long>(p.B) * p.Hq,
+                                                         (2LL * grid2 + nqb2 - 1) / nqb2));
+  k2<<<dim3(grid2), DqCfg<D>::kThreads, DqCfg<D>::kSmemAlloc, stream>>>(
       a.mq, a.mk, a.mv, a.mdo, a.mdq, a.L, a.Dv, static_cast<__nv_bfloat16*>(a.dq), p.Hq, group,
-      p.geom, Npad, scale_log2, p.scale, p.mask.win, p.cap);
+      p.geom, Npad, scale_log2, p.scale, p.mask.win, p.cap, a.sched + 1, static_cast<int>(g2),
+      tail2);
   p2.end();
   if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "bwd dQ launch");
   return ATTN_OK;
@@ -461,10 +475,10 @@ __global__ void selftest_wait_timeout_kernel() {
 // Backing store for attn_bwd_noalloc: the backward's lse*log2(e) and
 // rowsum(dO*O) rows live in this fixed device array instead of a
 // caller-provided workspace. Every device that loads the library holds these
-// 8 MiB until the process exits. Host code must not hand the symbol itself to
+// 8 MiB + 64 bytes until the process exits. Host code must not hand the symbol itself to
 // a kernel (on the host it names a stand-in, not device memory). Its device
 // address is looked up once per device with cudaGetSymbolAddress.
-constexpr size_t kStaticScratchBytes = size_t(8) << 20;
+constexpr size_t kStaticScratchBytes = (size_t(8) << 20) + attn::kBwdCounterBytes;
 static __device__ __align__(256) float g_bwd_scratch[kStaticScratchBytes / sizeof(float)];
 
 std::mutex g_scratch_mu;
@@ -693,7 +707,8 @@ attn_status bwd_run(const void* q, const void* k, const void* v, const void* o,
     return fail(ATTN_ERR_ARG,
                 "attn_bwd_noalloc: this shape needs %zu bytes of scratch, but the static area "
                 "holds %zu (B*Hq*ceil128(N) must be <= %zu); use attn_bwd with a workspace",
-                need, kStaticScratchBytes, kStaticScratchBytes / (2 * sizeof(float)));
+                need, kStaticScratchBytes,
+                (kStaticScratchBytes - attn::kBwdCounterBytes) / (2 * sizeof(float)));
   if (work && !use_static && workspace_bytes < need)
     return fail(ATTN_ERR_ARG, "workspace is %zu bytes, needs %zu", workspace_bytes, need);
   if ((st = ensure_init()) != ATTN_OK) return st;
@@ -726,6 +741,7 @@ attn_status bwd_run(const void* q, const void* k, const void* v, const void* o,
   a.o = o; a.lse = lse; a.dO = dO; a.dq = dq; a.dk = dk; a.dv = dv;
   a.L = static_cast<float*>(scratch);
   a.Dv = a.L + static_cast<size_t>(p.B) * p.Hq * attn::pad128(p.geom.Nq);
+  a.sched = reinterpret_cast<int*>(a.Dv + static_cast<size_t>(p.B) * p.Hq * attn::pad128(p.geom.Nq));
   if (p.d == 64) return dispatch_bwd<64>(a, p, stream);
   return dispatch_bwd<128>(a, p, stream);
 }
@@ -809,8 +825,9 @@ size_t attn_bwd_workspace_size(int B, int Hq, int N, int d) {
   (void)d;
   if (B <= 0 || Hq <= 0 || N <= 0) return 0;
   // lse * log2(e) and D = rowsum(dO * O), fp32, one row per query padded to
-  // a multiple of 128 per head.
-  return 2 * static_cast<size_t>(B) * Hq * attn::pad128(N) * sizeof(float);
+  // a multiple of 128 per head, then the persistent kernels' work counters.
+  return 2 * static_cast<size_t>(B) * Hq * attn::pad128(N) * sizeof(float) +
+         attn::kBwdCounterBytes;
 }
 
 attn_status attn_bwd(const void* q, const void* k, const void* v, const void* o,

@@ -90,12 +90,15 @@ attn_status attn_fwd(const void* q, const void* k, const void* v, void* o, float
  *        is the sum over the Hq/Hkv query heads that read it.
  *   workspace: caller-owned device scratch of at least
  *        attn_bwd_workspace_size(B, Hq, N, d) bytes, 16-byte aligned. Its
- *        contents on entry are ignored, and it is overwritten.
+ *        contents on entry are ignored, and it is overwritten. It must not be
+ *        shared by backward calls that can overlap on the GPU.
  * The pages do not write out the backward math. It is the exact gradient of
  * the forward definition: dV = P^T dO, dS = P * (dP - rowsum(dO * O)) with
  * dP = dO V^T, dQ = scale * dS K, dK = scale * dS^T Q. The P used is
  * recomputed from q, k and lse, so no N x N matrix is stored. The result is
- * deterministic: no atomics, the same bits on every run.
+ * deterministic, the same bits on every run: each gradient tile is computed
+ * by one CTA alone (the only atomics hand out work items, which does not
+ * change what any item computes).
  */
 attn_status attn_bwd(const void* q, const void* k, const void* v, const void* o,
                      const float* lse, const void* dO, void* dq, void* dk, void* dv,
@@ -106,8 +109,9 @@ attn_status attn_bwd(const void* q, const void* k, const void* v, const void* o,
  * Bytes of workspace attn_bwd needs for this shape (0 for an empty problem).
  * The pages have no counterpart: it exists because this library never
  * allocates, so the caller sizes and owns the backward's scratch (two fp32
- * rows per query, padded to a multiple of 128 per head). d is accepted for
- * symmetry with the other calls and does not change the size.
+ * rows per query, padded to a multiple of 128 per head, and 64 bytes of work
+ * counters). d is accepted for symmetry with the other calls and does not
+ * change the size.
  */
 size_t attn_bwd_workspace_size(int B, int Hq, int N, int d);
 
@@ -119,11 +123,11 @@ size_t attn_bwd_workspace_size(int B, int Hq, int N, int d);
  * processes that place all device memory at start-up under a fixed budget.
  * Such callers cannot supply attn_bwd's workspace. This entry point takes the
  * same tensors as attn_bwd (inputs and outputs are still caller-owned) and
- * keeps its scratch in a fixed 8 MiB array that the library places in device
+ * keeps its scratch in a fixed array of 8 MiB + 64 bytes that the library places in device
  * memory. Every GPU that loads the library holds that array until the process
  * exits. The pages describe no such entry point. It has no counterpart there.
- *   - Limit: attn_bwd_workspace_size(B, Hq, N, d) must not exceed 8 MiB
- *     (8388608 bytes), i.e. B * Hq * (N rounded up to a multiple of 128)
+ *   - Limit: attn_bwd_workspace_size(B, Hq, N, d) must not exceed 8 MiB + 64
+ *     bytes (8388672 bytes), i.e. B * Hq * (N rounded up to a multiple of 128)
  *     <= 1048576. Larger shapes return ATTN_ERR_ARG with a message, and
  *     nothing is launched.
  *   - It calls no cudaMalloc, cudaFree or other allocating routine. The first
