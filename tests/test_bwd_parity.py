@@ -88,6 +88,34 @@ def test_bwd_c5_full_size_sampled_heads():
         assert torch.isfinite(g.float()).all()
 
 
+def test_bwd_workspace_contents_ignored():
+    """The backward's workspace (the lse/D rows and the work counters that the
+    persistent dK/dV and dQ kernels hand items out from) may hold anything on
+    entry: a workspace of 0xFF bytes (counters at -1), reused twice in a row,
+    gives the same gradients bit for bit as a zeroed one. The shape has more
+    work items than SMs (dK/dV: 4 x 4 x 18 = 288, dQ: 4 x 16 x 18 = 1152), so
+    the CTAs take items from the counters; two heads are checked against the
+    oracle as well."""
+    w = workloads.small("bwd_persistent", 4, 16, 4, 2304, 64, True, seed=41)
+    q, k, v, do = workloads.make_inputs(w)
+    qd, kd, vd, dod = to_dev(q, k, v, do)
+    o, lse = ea.attn_fwd(qd, kd, vd, scale=w.scale, causal=True)
+    need = ea.attn_bwd_workspace_size(w.B, w.Hq, w.N, w.d)
+    clean = torch.zeros(need, dtype=torch.uint8, device="cuda")
+    ref = ea.attn_bwd(qd, kd, vd, o, lse, dod, workspace=clean, scale=w.scale, causal=True)
+    dirty = torch.full((need,), 0xFF, dtype=torch.uint8, device="cuda")
+    for _ in range(2):
+        got = ea.attn_bwd(qd, kd, vd, o, lse, dod, workspace=dirty, scale=w.scale, causal=True)
+        ea.attn_check_status()
+        for x, y in zip(got, ref):
+            assert torch.equal(x, y)
+    # The oracle computes the listed KV heads and every query head of their groups.
+    kv_picks = [(0, 0), (w.B - 1, w.Hkv - 1)]
+    refs = oracle.attention_backward(q, k, v, do, w.scale, True, heads=kv_picks)
+    heads = {"dq": [(0, 0), (w.B - 1, w.Hq - 1)], "dk": kv_picks, "dv": kv_picks}
+    assert_grads_close(ref, refs, w.name, heads=heads)
+
+
 def test_bwd_deterministic():
     w = workloads.small("bwd_det", 2, 4, 2, 640, 128, True, seed=5)
     q, k, v, do = workloads.make_inputs(w)
