@@ -331,14 +331,31 @@ struct Problem {
   attn::Softcap cap;
 };
 
-// Heads per group of the forward's grid order for unmasked problems:
-// consecutive (batch, query head) indices whose K and V together stay well
-// inside L2 (about 48 MB of the 126 MB), rounded down to whole GQA groups.
-// Masked problems (causal, windows) use one group, to keep the heaviest blocks
-// of every head first. Measured on B200 (c3, N 4096 d 128): unmasked 1076 ->
-// 1137-1155 TFLOP/s with groups; causal within 1 %, and 2-4 % slower at N 2048.
-int fwd_head_group(const Problem& p) {
+// Heads per group of the forward's grid order (the list is walked group by
+// group, heaviest block first within a group).
+// - Unmasked: consecutive (batch, query head) indices whose K and V together
+//   stay well inside L2 (about 48 MB of the 126 MB), rounded down to whole GQA
+//   groups. Measured on B200 (c3, N 4096 d 128): 1076 -> 1137-1155 TFLOP/s.
+// - Causal: the smallest group whose block count is a whole number of snake
+//   periods (2 x grid entries), so the heavy-to-light order of each group
+//   balances the CTAs by itself, if its K and V fit in 80 MB; else one group.
+//   An L2-sized group that broke the periods was slower (c3 1012 -> 913); the
+//   aligned one is faster (c3 1021 -> 1044, c5 851 -> 861 TFLOP/s).
+// - Other masks (windows): one group.
+int fwd_head_group(const Problem& p, int nmb, int grid) {
   const long long all = static_cast<long long>(p.B) * p.Hq;
+  if (p.mask.mode == attn::kMaskCausal) {
+    long long a = 2LL * grid, b = nmb;     // a = gcd(2 grid, nmb) after the loop
+    while (b) {
+      const long long t = a % b;
+      a = b;
+      b = t;
+    }
+    const long long hg = 2LL * grid / a;   // >= 1, and hg * nmb is a multiple of 2 grid
+    const double kv_bytes_per_head = 2.0 * p.geom.Nk * p.d * 2.0 / (p.Hq / p.Hkv);
+    if (hg < all && hg * kv_bytes_per_head <= 80.0 * (1 << 20)) return static_cast<int>(hg);
+    return static_cast<int>(all);
+  }
   if (p.mask.mode != attn::kMaskNone) return static_cast<int>(all);
   const int group = p.Hq / p.Hkv;
   const double kv_bytes_per_head = 2.0 * p.geom.Nk * p.d * 2.0 / group;
@@ -372,8 +389,9 @@ attn_status launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUten
   const long long pairs = static_cast<long long>(p.B) * p.Hq * ((p.geom.Nq + 255) / 256);
   sched.one_tile = pairs < sm_count() ? 1 : 0;
   sched.nmb = sched.one_tile ? (p.geom.Nq + 127) / 128 : (p.geom.Nq + 255) / 256;
-  sched.hg = fwd_head_group(p);
   sched.total = static_cast<long long>(sched.BH) * sched.nmb;
+  sched.hg = fwd_head_group(p, sched.nmb,
+                            static_cast<int>(std::min<long long>(sched.total, sm_count())));
   if (sched.total > 0x7FFFFFFFLL) return fail(ATTN_ERR_ARG, "problem too large for one launch");
   dim3 grid(static_cast<unsigned>(std::min<long long>(sched.total, sm_count())));
   const float scale_log2 = p.scale * 1.4426950408889634f;
