@@ -190,8 +190,67 @@ def _check_dtype(t, dtype, name):
         raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
 
 
+# Per-step fast path of attn_fwd / attn_bwd. After one call has gone through
+# the full checks (which also loads the library and caches torch's device and
+# stream getters), calls whose tensors are plainly valid (exact torch.Tensor,
+# expected shapes and dtypes, contiguous, all on the current device) skip the
+# Python-side helpers and are marshalled by the _pycall module when it is
+# built (ctypes otherwise). Anything else takes the checked path, which raises
+# the specific error. The library repeats every check that matters for safety.
+_FAST = None      # (library handle, Tensor type, bf16, fp32, fwd caller, bwd caller)
+
+
+def _enable_fast():
+    global _FAST
+    import torch
+    lib = _lib
+    if lib is None or _GET_DEVICE is None or _RAW_STREAM is None:
+        return
+    try:
+        from . import _pycall
+    except ImportError:
+        _pycall = None
+    if _pycall is not None:
+        fa = ctypes.cast(lib.attn_fwd, ctypes.c_void_p).value
+        ba = ctypes.cast(lib.attn_bwd, ctypes.c_void_p).value
+        cf, cb = _pycall.call_fwd, _pycall.call_bwd
+        fwd = lambda *a: cf(fa, *a)  # noqa: E731
+        bwd = lambda *a: cb(ba, *a)  # noqa: E731
+    else:
+        fwd, bwd = lib.attn_fwd, lib.attn_bwd
+    _FAST = (lib, torch.Tensor, torch.bfloat16, torch.float32, fwd, bwd)
+
+
 def attn_fwd(q, k, v, o=None, lse=None, scale=None, causal=False, stream=None):
     """Forward pass; returns (o, lse). Allocates o/lse with torch if not given."""
+    fast = _FAST
+    if fast is not None and fast[0] is _lib:
+        T = fast[1]
+        if type(q) is T and type(k) is T and type(v) is T and type(o) is T and type(lse) is T:
+            qs, ks = q.shape, k.shape
+            if len(qs) == 4 and len(ks) == 4:
+                B, Hq, N, d = qs
+                bf = fast[2]
+                dev = q.get_device()
+                if (ks[0] == B and ks[2] == N and ks[3] == d and v.shape == ks and o.shape == qs
+                        and lse.shape == (B, Hq, N) and q.dtype is bf and k.dtype is bf
+                        and v.dtype is bf and o.dtype is bf and lse.dtype is fast[3] and dev >= 0
+                        and dev == _GET_DEVICE() and k.get_device() == dev
+                        and v.get_device() == dev and o.get_device() == dev
+                        and lse.get_device() == dev and q.is_contiguous() and k.is_contiguous()
+                        and v.is_contiguous() and o.is_contiguous() and lse.is_contiguous()):
+                    st = fast[4](q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
+                                 lse.data_ptr(), B, Hq, ks[1], N, d,
+                                 1.0 / math.sqrt(d) if scale is None else float(scale),
+                                 1 if causal else 0,
+                                 _RAW_STREAM(dev) if stream is None else stream.cuda_stream)
+                    if st != ATTN_OK:
+                        _check(st)
+                    return o, lse
+    return _attn_fwd_checked(q, k, v, o, lse, scale, causal, stream)
+
+
+def _attn_fwd_checked(q, k, v, o, lse, scale, causal, stream):
     import torch
     B, Hq, N, d = q.shape
     Hkv = k.shape[1]
@@ -217,6 +276,8 @@ def attn_fwd(q, k, v, o=None, lse=None, scale=None, causal=False, stream=None):
         _check(lib.attn_fwd(_dev_ptr(q, "q"), _dev_ptr(k, "k"), _dev_ptr(v, "v"), _dev_ptr(o, "o"),
                             _dev_ptr(lse, "lse"), B, Hq, Hkv, N, d, scale, int(bool(causal)),
                             g.stream(stream)))
+    if _FAST is None or _FAST[0] is not _lib:
+        _enable_fast()
     return o, lse
 
 
@@ -260,6 +321,36 @@ def _check_grad_outputs(dq, dk, dv, q, k, v):
 def attn_bwd(q, k, v, o, lse, dO, dq=None, dk=None, dv=None, workspace=None, scale=None,
              causal=False, stream=None):
     """Backward pass; returns (dq, dk, dv). Allocates outputs/workspace if not given."""
+    fast = _FAST
+    if (fast is not None and fast[0] is _lib and type(q) is fast[1] and type(k) is fast[1]
+            and type(lse) is fast[1] and type(workspace) is fast[1]):
+        T, bf = fast[1], fast[2]
+        qs, ks = q.shape, k.shape
+        if len(qs) == 4 and len(ks) == 4 and workspace.is_contiguous():
+            B, Hq, N, d = qs
+            dev = q.get_device()
+            ptrs = []
+            if (ks[0] == B and ks[2] == N and ks[3] == d and lse.shape == (B, Hq, N)
+                    and lse.dtype is fast[3] and dev >= 0 and dev == _GET_DEVICE()):
+                for t, shape in ((q, qs), (k, ks), (v, ks), (o, qs), (lse, None), (dO, qs),
+                                 (dq, qs), (dk, ks), (dv, ks)):
+                    if (type(t) is not T or t.get_device() != dev or not t.is_contiguous()
+                            or (shape is not None and (t.shape != shape or t.dtype is not bf))):
+                        break
+                    ptrs.append(t.data_ptr())
+            if len(ptrs) == 9 and workspace.get_device() == dev:
+                st = fast[5](*ptrs, workspace.data_ptr(),
+                             workspace.numel() * workspace.element_size(), B, Hq, ks[1], N, d,
+                             1.0 / math.sqrt(d) if scale is None else float(scale),
+                             1 if causal else 0,
+                             _RAW_STREAM(dev) if stream is None else stream.cuda_stream)
+                if st != ATTN_OK:
+                    _check(st)
+                return dq, dk, dv
+    return _attn_bwd_checked(q, k, v, o, lse, dO, dq, dk, dv, workspace, scale, causal, stream)
+
+
+def _attn_bwd_checked(q, k, v, o, lse, dO, dq, dk, dv, workspace, scale, causal, stream):
     import torch
     B, Hq, Hkv, N, d = _check_bwd_inputs(q, k, v, o, lse, dO)
     dq = torch.empty_like(q) if dq is None else dq
@@ -277,6 +368,8 @@ def attn_bwd(q, k, v, o, lse, dO, dq=None, dk=None, dv=None, workspace=None, sca
                             _dev_ptr(dk, "dk"), _dev_ptr(dv, "dv"), _dev_ptr(workspace, "workspace"),
                             workspace.numel() * workspace.element_size(),
                             B, Hq, Hkv, N, d, scale, int(bool(causal)), g.stream(stream)))
+    if _FAST is None or _FAST[0] is not _lib:
+        _enable_fast()
     return dq, dk, dv
 
 

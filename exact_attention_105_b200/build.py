@@ -2,8 +2,9 @@
 
 ``python -m exact_attention_105_b200.build`` (or ``build()``) compiles
 ``csrc/attn_api.cu``, the single translation unit that holds every kernel, into
-``libattn_sm100.so`` next to this file. It rebuilds only when a source is
-newer than the library.
+``libattn_sm100.so`` next to this file, and ``csrc/pycall.c`` (the CPython
+argument marshalling for the per-step calls) into ``_pycall`` with the host C
+compiler. Each rebuilds only when its sources are newer than its output.
 """
 from __future__ import annotations
 
@@ -11,12 +12,15 @@ import os
 import shutil
 import subprocess
 import sys
+import sysconfig
 
 HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(os.path.dirname(HERE), "include")
 LIB_NAME = "libattn_sm100.so"
 LIB_PATH = os.path.join(HERE, LIB_NAME)
+PYCALL_SRC = os.path.join(CSRC, "pycall.c")
+PYCALL_PATH = os.path.join(HERE, "_pycall" + (sysconfig.get_config_var("EXT_SUFFIX") or ".so"))
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",
@@ -48,10 +52,35 @@ def is_stale() -> bool:
     return any(os.path.getmtime(s) > lib_m for s in _sources())
 
 
+def build_pycall(force: bool = False) -> str:
+    """Compile the CPython marshalling module if needed; return its path."""
+    if (not force and os.path.exists(PYCALL_PATH)
+            and os.path.getmtime(PYCALL_PATH) >= os.path.getmtime(PYCALL_SRC)):
+        return PYCALL_PATH
+    cc = os.environ.get("CC") or shutil.which("gcc") or shutil.which("cc")
+    if not cc:
+        raise RuntimeError("no host C compiler (gcc/cc) for " + PYCALL_SRC)
+    tmp = PYCALL_PATH + ".tmp"
+    cmd = [cc, "-O2", "-shared", "-fPIC", "-I", sysconfig.get_paths()["include"], "-o", tmp,
+           PYCALL_SRC]
+    proc = subprocess.run(cmd, capture_output=True, text=True)
+    if proc.returncode != 0:
+        raise RuntimeError(f"{cc} failed ({proc.returncode}):\n{' '.join(cmd)}\n"
+                           f"{proc.stdout}{proc.stderr}")
+    os.replace(tmp, PYCALL_PATH)
+    return PYCALL_PATH
+
+
 def build(force: bool = False, verbose: bool = False) -> str:
-    """Compile the library if needed; return its path. Raises on failure."""
-    if not force and not is_stale():
-        return LIB_PATH
+    """Compile the library and the marshalling module if needed; return the
+    library's path. Raises on failure."""
+    if force or is_stale():
+        _build_library(verbose)
+    build_pycall(force)
+    return LIB_PATH
+
+
+def _build_library(verbose: bool) -> None:
     tmp = LIB_PATH + ".tmp"
     cmd = [_nvcc(), *NVCC_FLAGS, "-o", tmp, os.path.join(CSRC, "attn_api.cu")]
     proc = subprocess.run(cmd, cwd=CSRC, capture_output=True, text=True)
@@ -63,7 +92,6 @@ def build(force: bool = False, verbose: bool = False) -> str:
     os.replace(tmp, LIB_PATH)
     with open(os.path.join(HERE, "ptxas_info.txt"), "w") as f:
         f.write(log)
-    return LIB_PATH
 
 
 if __name__ == "__main__":

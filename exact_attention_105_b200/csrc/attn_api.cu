@@ -13,7 +13,9 @@
 #include <cstdio>
 #include <cstring>
 #include <algorithm>
+#include <atomic>
 #include <mutex>
+#include <utility>
 #include <vector>
 
 #include "../../include/attn.h"
@@ -105,9 +107,21 @@ std::once_flag g_init_once;
 constexpr int kMaxDevices = 64;
 int g_sm_count[kMaxDevices] = {};             // multiprocessors, filled by check_device()
 
-int sm_count() {
+// The device current for the API call this thread is in. check_device(),
+// which every entry point runs before anything that needs the device, sets
+// it, so the rest of the call does not query the runtime again.
+thread_local int t_call_dev = -1;
+
+int call_device() {
+  if (t_call_dev >= 0) return t_call_dev;
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 148;
+  if (cudaGetDevice(&dev) != cudaSuccess) return -1;
+  return dev;
+}
+
+int sm_count() {
+  const int dev = call_device();
+  if (dev < 0 || dev >= kMaxDevices) return 148;
   return g_sm_count[dev] > 0 ? g_sm_count[dev] : 148;
 }
 
@@ -126,6 +140,7 @@ void init_once() {
 
 // The current device must be an sm_100 part; checked once per device.
 attn_status check_device() {
+  t_call_dev = -1;
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) {
@@ -133,22 +148,31 @@ attn_status check_device() {
     return fail(ATTN_ERR_CUDA, "no CUDA device: %s", cudaGetErrorString(e));
   }
   if (dev < 0 || dev >= kMaxDevices) return fail(ATTN_ERR_CUDA, "device index %d unsupported", dev);
+  // 0: not checked yet, else major * 10 + minor. Written once per device
+  // under the mutex (after g_sm_count), read without it afterwards.
   static std::mutex mu;
-  static int arch[kMaxDevices] = {};          // 0: not checked yet, else major * 10 + minor
-  std::lock_guard<std::mutex> g(mu);
-  if (arch[dev] == 0) {
-    cudaDeviceProp prop;
-    e = cudaGetDeviceProperties(&prop, dev);
-    if (e != cudaSuccess) {
-      cudaGetLastError();
-      return fail(ATTN_ERR_CUDA, "cudaGetDeviceProperties(%d): %s", dev, cudaGetErrorString(e));
+  static std::atomic<int> arch[kMaxDevices] = {};
+  int a = arch[dev].load(std::memory_order_acquire);
+  if (a == 0) {
+    std::lock_guard<std::mutex> g(mu);
+    a = arch[dev].load(std::memory_order_relaxed);
+    if (a == 0) {
+      cudaDeviceProp prop;
+      e = cudaGetDeviceProperties(&prop, dev);
+      if (e != cudaSuccess) {
+        cudaGetLastError();
+        return fail(ATTN_ERR_CUDA, "cudaGetDeviceProperties(%d): %s", dev,
+                    cudaGetErrorString(e));
+      }
+      g_sm_count[dev] = prop.multiProcessorCount;
+      a = prop.major * 10 + prop.minor;
+      arch[dev].store(a, std::memory_order_release);
     }
-    arch[dev] = prop.major * 10 + prop.minor;
-    g_sm_count[dev] = prop.multiProcessorCount;
   }
-  if (arch[dev] != 100)
+  if (a != 100)
     return fail(ATTN_ERR_CUDA, "this library is built for sm_100a (B200); device %d is sm_%d", dev,
-                arch[dev]);
+                a);
+  t_call_dev = dev;
   return ATTN_OK;
 }
 
@@ -166,29 +190,52 @@ attn_status ensure_init() {
 // setmaxnreg split).
 struct KernelSetup {
   std::mutex mu;
-  bool done[kMaxDevices] = {};
+  std::atomic<bool> done[kMaxDevices] = {};   // set (release) after err and regs
   cudaError_t err[kMaxDevices] = {};
   int regs[kMaxDevices] = {};
 };
 
 template <typename Kern>
 cudaError_t prepare_kernel(Kern kern, int smem_bytes, KernelSetup& ks, int* regs = nullptr) {
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return e;
+  const int dev = call_device();
   if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
-  std::lock_guard<std::mutex> g(ks.mu);
-  if (!ks.done[dev]) {
-    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes);
-    cudaFuncAttributes fa;
-    if (e == cudaSuccess) e = cudaFuncGetAttributes(&fa, kern);
-    ks.err[dev] = e;
-    ks.regs[dev] = (e == cudaSuccess) ? fa.numRegs : 0;
-    ks.done[dev] = true;
+  if (!ks.done[dev].load(std::memory_order_acquire)) {
+    std::lock_guard<std::mutex> g(ks.mu);
+    if (!ks.done[dev].load(std::memory_order_relaxed)) {
+      cudaError_t e =
+          cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes);
+      cudaFuncAttributes fa;
+      if (e == cudaSuccess) e = cudaFuncGetAttributes(&fa, kern);
+      ks.err[dev] = e;
+      ks.regs[dev] = (e == cudaSuccess) ? fa.numRegs : 0;
+      ks.done[dev].store(true, std::memory_order_release);
+    }
   }
   if (regs) *regs = ks.regs[dev];
   return ks.err[dev];
 }
+// Launch with programmatic stream serialization: the kernel may be launched
+// while the kernel before it on the stream finishes (every kernel here waits
+// for its predecessor with griddepcontrol.wait before touching global memory,
+// and allows its successor's launch once all its CTAs have finished their
+// work). Between two launches of this library that hides the launch latency
+// and the next kernel's set-up, which is what short problems are made of.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, int threads, int smem,
+                       cudaStream_t stream, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(static_cast<unsigned>(threads));
+  cfg.dynamicSmemBytes = static_cast<size_t>(smem);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
+
 // 3-D tensor map (d, rows, z) over a bf16 tensor, with a box of 64 x 128 x 1
 // (one 128-row, 128-byte-wide column block) and 128-byte swizzle. Row and z
 // strides are in elements. Fixed-length [B*H, N, d]: rows = N, z = B*H,
@@ -250,11 +297,10 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 // host pointer, or memory of another GPU than the current one, handed to a
 // kernel would fault the GPU, so both are rejected here.
 attn_status check_device_ptr(const void* ptr, const char* name) {
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  const int dev = call_device();
+  if (dev < 0) return fail(ATTN_ERR_CUDA, "cudaGetDevice failed");
   cudaPointerAttributes pa;
-  e = cudaPointerGetAttributes(&pa, ptr);
+  cudaError_t e = cudaPointerGetAttributes(&pa, ptr);
   if (e != cudaSuccess) {
     cudaGetLastError();
     return fail(ATTN_ERR_ARG, "%s is not a CUDA pointer (%s)", name, cudaGetErrorName(e));
@@ -396,12 +442,14 @@ attn_status launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUten
   dim3 grid(static_cast<unsigned>(std::min<long long>(sched.total, sm_count())));
   const float scale_log2 = p.scale * 1.4426950408889634f;
   ProfScope ps(kProfFwd, stream);
-  kern<<<grid, Cfg::kThreads, Cfg::kSmemAlloc, stream>>>(
-      mq, mk, mv, mo, static_cast<__nv_bfloat16*>(o), lse, p.Hq, p.Hq / p.Hkv, p.geom, scale_log2,
-      p.mask.win, p.cap, sched);
+  cudaError_t e = launch_pdl(kern, grid, Cfg::kThreads, Cfg::kSmemAlloc, stream, mq, mk, mv, mo,
+                             static_cast<__nv_bfloat16*>(o), lse, p.Hq, p.Hq / p.Hkv, p.geom,
+                             scale_log2, p.mask.win, p.cap, sched);
   ps.end();
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return cuda_fail(e, "fwd kernel launch");
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return cuda_fail(e, "fwd kernel launch");
+  }
   return ATTN_OK;
 }
 
@@ -429,12 +477,15 @@ attn_status launch_bwd(const BwdArgs& a, const Problem& p, cudaStream_t stream) 
   if (rows / 32 > 0x7FFFFFFFLL || g1 > 0x7FFFFFFFLL || g2 > 0x7FFFFFFFLL)
     return fail(ATTN_ERR_ARG, "problem too large for one launch");
   ProfScope p0(kProfBwdPre, stream);
-  bwd_pre_kernel<D><<<static_cast<unsigned>(rows / 32), 256, 0, stream>>>(
-      static_cast<const __nv_bfloat16*>(a.o), static_cast<const __nv_bfloat16*>(a.dO), a.lse,
-      a.L, a.Dv, p.Hq, p.geom, Npad, a.sched);
+  cudaError_t e = launch_pdl(bwd_pre_kernel<D>, dim3(static_cast<unsigned>(rows / 32)), 256, 0,
+                             stream, static_cast<const __nv_bfloat16*>(a.o),
+                             static_cast<const __nv_bfloat16*>(a.dO), a.lse, a.L, a.Dv, p.Hq,
+                             p.geom, Npad, a.sched);
   p0.end();
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return cuda_fail(e, "bwd preprocess launch");
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return cuda_fail(e, "bwd preprocess launch");
+  }
 
   static KernelSetup s1, s2;
   auto k1 = bwd_dkdv_kernel<D, MODE, FEAT>;
@@ -451,24 +502,30 @@ attn_status launch_bwd(const BwdArgs& a, const Problem& p, cudaStream_t stream) 
   const int nkv1 = pad128(p.geom.Nk) / 128;
   const int tail1 = static_cast<int>(std::min<long long>(static_cast<long long>(p.B) * p.Hkv,
                                                          (2LL * grid1 + nkv1 - 1) / nkv1));
-  k1<<<dim3(grid1), DkdvCfg<D>::kThreads, DkdvCfg<D>::kSmemAlloc, stream>>>(
-      a.mq, a.mk, a.mv, a.mdo, a.mdk, a.mdv, a.L, a.Dv, static_cast<__nv_bfloat16*>(a.dk),
-      static_cast<__nv_bfloat16*>(a.dv), p.Hq, group, p.geom, Npad, scale_log2, p.scale,
-      p.mask.win, p.cap, a.sched, static_cast<int>(g1), tail1);
+  e = launch_pdl(k1, dim3(grid1), DkdvCfg<D>::kThreads, DkdvCfg<D>::kSmemAlloc, stream, a.mq,
+                 a.mk, a.mv, a.mdo, a.mdk, a.mdv, a.L, a.Dv, static_cast<__nv_bfloat16*>(a.dk),
+                 static_cast<__nv_bfloat16*>(a.dv), p.Hq, group, p.geom, Npad, scale_log2,
+                 p.scale, p.mask.win, p.cap, a.sched, static_cast<int>(g1), tail1);
   p1.end();
-  if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "bwd dK/dV launch");
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return cuda_fail(e, "bwd dK/dV launch");
+  }
   ProfScope p2(kProfBwdDq, stream);
   // dQ work items: (batch, query head, 128-query block); persistent as above.
   const unsigned grid2 = static_cast<unsigned>(std::min<long long>(g2, sm_count()));
   const int nqb2 = Npad / 128;
   const int tail2 = static_cast<int>(std::min<long long>(static_cast<long long>(p.B) * p.Hq,
                                                          (2LL * grid2 + nqb2 - 1) / nqb2));
-  k2<<<dim3(grid2), DqCfg<D>::kThreads, DqCfg<D>::kSmemAlloc, stream>>>(
-      a.mq, a.mk, a.mv, a.mdo, a.mdq, a.L, a.Dv, static_cast<__nv_bfloat16*>(a.dq), p.Hq, group,
-      p.geom, Npad, scale_log2, p.scale, p.mask.win, p.cap, a.sched + 1, static_cast<int>(g2),
-      tail2);
+  e = launch_pdl(k2, dim3(grid2), DqCfg<D>::kThreads, DqCfg<D>::kSmemAlloc, stream, a.mq, a.mk,
+                 a.mv, a.mdo, a.mdq, a.L, a.Dv, static_cast<__nv_bfloat16*>(a.dq), p.Hq, group,
+                 p.geom, Npad, scale_log2, p.scale, p.mask.win, p.cap, a.sched + 1,
+                 static_cast<int>(g2), tail2);
   p2.end();
-  if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "bwd dQ launch");
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return cuda_fail(e, "bwd dQ launch");
+  }
   return ATTN_OK;
 }
 

@@ -69,6 +69,7 @@ __global__ void __launch_bounds__(256)
 bwd_pre_kernel(const __nv_bfloat16* __restrict__ o, const __nv_bfloat16* __restrict__ dO,
                const float* __restrict__ lse, float* __restrict__ L, float* __restrict__ Dv,
                int Hq, SeqGeom geom, int Npad, int* __restrict__ sched) {
+  grid_dep_wait();     // o and lse may come from the kernel just before
   if (blockIdx.x == 0 && threadIdx.x < kBwdCounters) sched[threadIdx.x] = 0;
   const long long row = static_cast<long long>(blockIdx.x) * 32 + (threadIdx.x >> 3);
   const int sub = threadIdx.x & 7;
@@ -105,6 +106,7 @@ bwd_pre_kernel(const __nv_bfloat16* __restrict__ o, const __nv_bfloat16* __restr
     L[row] = (l == -INFINITY) ? -INFINITY : -l * kLog2e;
     Dv[row] = (n < N) ? -acc : 0.f;
   }
+  grid_dep_launch();
 }
 
 // ------------------------------------------------------------------ shared bits
@@ -337,6 +339,8 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  // Set-up done; the previous kernel's results must be visible from here on.
+  grid_dep_wait();
 
   // Item k of this CTA, as published by the producer (-1: no more).
   auto read_item = [&](int k, int& item) {
@@ -701,6 +705,7 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 
   tc_fence_before();
   __syncthreads();
+  grid_dep_launch();
   if (warp == 9) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
@@ -846,6 +851,8 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  // Set-up done; the previous kernel's results must be visible from here on.
+  grid_dep_wait();
 
   auto read_item = [&](int k, int& item) {
     if (!mbar_wait(&item_full[k % IS], (k / IS) & 1, abort_flag, kSiteBItem)) return false;
@@ -1205,6 +1212,7 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
 
   tc_fence_before();
   __syncthreads();
+  grid_dep_launch();
   if (warp == 9) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);

@@ -218,6 +218,8 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  // Set-up done; the previous kernel's results must be visible from here on.
+  grid_dep_wait();
 
   if (warp >= 8) {
     regs_shrink<kFwdRegsSmall>();
@@ -684,6 +686,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
 
   tc_fence_before();
   __syncthreads();
+  grid_dep_launch();
   if (warp == 9) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);

@@ -207,6 +207,23 @@ __device__ __forceinline__ void tc_fence_before() {
 __device__ __forceinline__ void tc_fence_after() {
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 }
+
+// Programmatic dependent launch. The host launches every kernel of this
+// library with programmatic stream serialization, so a kernel may be launched
+// before the kernel ahead of it on the stream has completed. grid_dep_wait()
+// blocks until that kernel has completed and its memory writes are visible;
+// every thread calls it before its first global-memory access (the set-up of
+// barriers and tensor memory comes before it). grid_dep_launch() allows the
+// next kernel's launch once every CTA of this grid has issued it or exited.
+// The kernels issue it when a CTA's work is done, just before tensor memory
+// is released: issued at the start instead, the next grid's CTAs took SMs
+// while this grid was still running and the large problems ran 1-2 % slower.
+__device__ __forceinline__ void grid_dep_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+__device__ __forceinline__ void grid_dep_launch() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
 // Arrive once on `bar` when every tcgen05 async op issued so far by this
 // thread has completed.
 __device__ __forceinline__ void tc_commit(uint64_t* bar) {

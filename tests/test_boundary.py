@@ -105,6 +105,31 @@ def test_bwd_argument_errors(lib, kw, code):
     assert bwd(lib, **kw) == code
 
 
+def test_marshalling_module_calls_the_library(lib):
+    """_pycall converts the ints and floats the binding passes and calls the
+    function at the address it is given. With arguments the library rejects
+    before touching a device, the library's status and message come back."""
+    from exact_attention_105_b200 import _pycall
+    fa = ctypes.cast(lib.attn_fwd, ctypes.c_void_p).value
+    ba = ctypes.cast(lib.attn_bwd, ctypes.c_void_p).value
+    assert _pycall.call_fwd(fa, FAKE, FAKE, FAKE, FAKE, FAKE, 1, 3, 2, 128, 64, 0.125, 0,
+                            None) == ea.ATTN_ERR_ARG
+    assert "divisible" in lib.attn_get_last_error().decode()
+    assert _pycall.call_fwd(fa, FAKE, FAKE, FAKE, FAKE, FAKE, 1, 2, 1, 128, 64, 0.125, 2,
+                            None) == ea.ATTN_ERR_ARG
+    assert "causal" in lib.attn_get_last_error().decode()
+    assert _pycall.call_bwd(ba, *([FAKE] * 10), 1 << 30, 1, 2, 1, 128, 96, 0.125, 0,
+                            None) == ea.ATTN_ERR_UNSUPPORTED
+    assert _pycall.call_bwd(ba, *([FAKE] * 10), 1 << 30, 1, 2, 1, 128, 64, 0.125, 0,
+                            None) in (ea.ATTN_ERR_ARG, ea.ATTN_ERR_CUDA)
+    with pytest.raises(TypeError):
+        _pycall.call_fwd(fa, FAKE)
+    with pytest.raises(OverflowError):
+        _pycall.call_fwd(fa, FAKE, FAKE, FAKE, FAKE, FAKE, 1 << 40, 2, 1, 128, 64, 0.125, 0, None)
+    with pytest.raises(ValueError):
+        _pycall.call_fwd(0, FAKE, FAKE, FAKE, FAKE, FAKE, 1, 2, 1, 128, 64, 0.125, 0, None)
+
+
 def test_workspace_size(lib):
     assert lib.attn_bwd_workspace_size(0, 4, 128, 64) == 0
     small = lib.attn_bwd_workspace_size(1, 1, 128, 64)

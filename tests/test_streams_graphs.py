@@ -73,6 +73,50 @@ def test_two_streams_at_once():
         assert torch.equal(got, want)
 
 
+def test_fast_and_checked_paths_agree():
+    """Calls with their outputs passed in take the per-step path once a fully
+    checked call has run. Its results are bitwise those of the checked path,
+    on the current stream and on a given one, and arguments it cannot vouch
+    for still get the checked path's errors."""
+    q, k, v, do = _problem(7)
+    shape_lse = q.shape[:3]
+    ws = torch.empty(ea.attn_bwd_workspace_size(2, 4, 700, 128), dtype=torch.uint8, device="cuda")
+
+    def outputs():
+        return (torch.empty_like(q), torch.empty(shape_lse, device="cuda"), torch.empty_like(q),
+                torch.empty_like(k), torch.empty_like(v))
+
+    o1, lse1, dq1, dk1, dv1 = outputs()
+    ea._attn_fwd_checked(q, k, v, o1, lse1, None, True, None)
+    ea._attn_bwd_checked(q, k, v, o1, lse1, do, dq1, dk1, dv1, ws, None, True, None)
+    assert ea._FAST is not None and ea._FAST[0] is ea.load_library()
+    o2, lse2, dq2, dk2, dv2 = outputs()
+    ea.attn_fwd(q, k, v, o2, lse2, causal=True)
+    ea.attn_bwd(q, k, v, o2, lse2, do, dq2, dk2, dv2, ws, causal=True)
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    o3, lse3, dq3, dk3, dv3 = outputs()
+    ea.attn_fwd(q, k, v, o3, lse3, causal=True, stream=s)
+    ea.attn_bwd(q, k, v, o3, lse3, do, dq3, dk3, dv3, ws, causal=True, stream=s)
+    s.synchronize()
+    torch.cuda.synchronize()
+    ea.attn_check_status()
+    for got2, got3, want in zip((o2, lse2, dq2, dk2, dv2), (o3, lse3, dq3, dk3, dv3),
+                                (o1, lse1, dq1, dk1, dv1)):
+        assert torch.equal(got2, want)
+        assert torch.equal(got3, want)
+    o_t = torch.empty(q.shape[0], q.shape[2], q.shape[1], q.shape[3], dtype=q.dtype,
+                      device="cuda").transpose(1, 2)
+    with pytest.raises(ValueError, match="contiguous"):
+        ea.attn_fwd(q, k, v, o_t, lse2, causal=True)
+    with pytest.raises(TypeError, match="lse must be"):
+        ea.attn_fwd(q, k, v, o2, lse2.double(), causal=True)
+    with pytest.raises(ValueError, match="shape"):
+        ea.attn_fwd(q, k, v[:, :, :600], o2, lse2, causal=True)
+    with pytest.raises(TypeError, match="dq must be"):
+        ea.attn_bwd(q, k, v, o2, lse2, do, dq2.float(), dk2, dv2, ws, causal=True)
+
+
 def test_calls_from_several_host_threads():
     problems = [_problem(10 + i, N=300 + 200 * i) for i in range(4)]
     refs = [_eager(*p) for p in problems]
