@@ -14,7 +14,9 @@
 #include <cstring>
 #include <algorithm>
 #include <atomic>
+#include <memory>
 #include <mutex>
+#include <queue>
 #include <utility>
 #include <vector>
 
@@ -411,12 +413,144 @@ int fwd_head_group(const Problem& p, int nmb, int grid) {
   return static_cast<int>(std::min<long long>(hg, all));
 }
 
-template <int D, int MODE, int FEAT>
-attn_status launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
-                       const CUtensorMap& mo, void* o, float* lse, const Problem& p,
-                       cudaStream_t stream) {
+// ---------------------------------------------------------------- causal plan
+// Causal blocks differ in cost: block mb of a head has about 2 mb + 2 key-tile
+// steps. When the block count is not a whole number of snake periods, the
+// snake leaves some CTAs with much more work than others (c5, 1024 blocks on
+// 148 CTAs: 54 to 70 steps, 62.3 on average). The plan instead hands each list
+// entry, in list order, to the CTA with the least work so far, costed as its
+// key-tile steps plus kPlanBlockCost steps for the block's start and end (clock
+// stamps: a 256-row block pays about 2.5 us at its boundary, a step about 1.9
+// us). It keeps the list order, so heads still come in groups that fit L2.
+
+constexpr double kPlanBlockCost = 1.3;
+
+// The list entries' costs for a causal fixed-length problem, in list order
+// (the same decoding as fwd_block).
+std::vector<double> causal_costs(const attn::FwdSched& sc, int N) {
+  std::vector<double> cost(static_cast<size_t>(sc.total));
+  const int rb = sc.one_tile ? 128 : 256;
+  const long long per_group = static_cast<long long>(sc.hg) * sc.nmb;
+  for (long long idx = 0; idx < sc.total; ++idx) {
+    const long long g = idx / per_group, r = idx - g * per_group;
+    const long long gs = std::min<long long>(sc.hg, sc.BH - g * sc.hg);
+    const int mb = sc.nmb - 1 - static_cast<int>(r / gs);
+    const int m0 = mb * rb;
+    int lo = 0, hi = -1;
+    attn::kv_tile_range<attn::kMaskCausal>(m0, std::min(m0 + rb - 1, N - 1), N, attn::KeyWindow{},
+                                           lo, hi);
+    cost[static_cast<size_t>(idx)] = (hi - lo + 1) + kPlanBlockCost;
+  }
+  return cost;
+}
+
+// Largest per-CTA cost of the snake assignment.
+double snake_makespan(const std::vector<double>& cost, int grid) {
+  std::vector<double> load(static_cast<size_t>(grid), 0.0);
+  for (size_t idx = 0; idx < cost.size(); ++idx) {
+    const size_t t = idx / grid, c = idx % grid;
+    load[(t & 1) ? grid - 1 - c : c] += cost[idx];
+  }
+  return *std::max_element(load.begin(), load.end());
+}
+
+// List scheduling in list order onto the least-loaded CTA (lowest index on
+// ties). Fills `owner` and returns the largest per-CTA cost.
+double list_schedule(const std::vector<double>& cost, int grid, std::vector<int>* owner) {
+  using Slot = std::pair<double, int>;
+  std::priority_queue<Slot, std::vector<Slot>, std::greater<Slot>> heap;
+  for (int c = 0; c < grid; ++c) heap.push({0.0, c});
+  double makespan = 0.0;
+  if (owner) owner->resize(cost.size());
+  for (size_t idx = 0; idx < cost.size(); ++idx) {
+    Slot sl = heap.top();
+    heap.pop();
+    sl.first += cost[idx];
+    makespan = std::max(makespan, sl.first);
+    if (owner) (*owner)[idx] = sl.second;
+    heap.push(sl);
+  }
+  return makespan;
+}
+
+struct PlanKey {
+  long long total;
+  int BH, nmb, one_tile, N, grid, group;
+  double kv_head;
+  bool operator==(const PlanKey& o) const {
+    return total == o.total && BH == o.BH && nmb == o.nmb && one_tile == o.one_tile &&
+           N == o.N && grid == o.grid && group == o.group && kv_head == o.kv_head;
+  }
+};
+struct PlanEntry {
+  PlanKey key;
+  std::shared_ptr<const attn::FwdPlan> plan;   // null: the snake is as good
+  int hg;
+};
+std::mutex g_plan_mu;
+std::vector<PlanEntry> g_plans;                // a few recent shapes, newest last
+
+// The plan for a causal fixed-length problem, or null when the snake is within
+// 2 % of it. Head groups: the sizes that divide the heads evenly (whole GQA
+// groups) with K and V of at most 48 MB, the one with the smallest planned
+// makespan. Sets sc->hg to the group size the returned plan (or the snake)
+// uses. Cached per shape.
+std::shared_ptr<const attn::FwdPlan> causal_plan(const Problem& p, int grid, attn::FwdSched* sc) {
+  const int group = p.Hq / p.Hkv;
+  const double kv_head = 2.0 * p.geom.Nk * p.d * 2.0 / group;
+  const PlanKey key{sc->total, sc->BH, sc->nmb, sc->one_tile, p.geom.Nq, grid, group, kv_head};
+  {
+    std::lock_guard<std::mutex> g(g_plan_mu);
+    for (const PlanEntry& e : g_plans)
+      if (e.key == key) {
+        sc->hg = e.hg;
+        return e.plan;
+      }
+  }
+  const double snake = snake_makespan(causal_costs(*sc, p.geom.Nq), grid);
+  const int snake_hg = sc->hg;
+  int best_hg = 0;
+  double best = 0.0;
+  for (int hg = group; hg <= sc->BH; hg += group) {
+    if (sc->BH % hg != 0 || (hg > group && hg * kv_head > 48.0 * (1 << 20))) continue;
+    sc->hg = hg;
+    const double m = list_schedule(causal_costs(*sc, p.geom.Nq), grid, nullptr);
+    if (best_hg == 0 || m < best * 0.999) {
+      best = m;
+      best_hg = hg;
+    }
+  }
+  std::shared_ptr<attn::FwdPlan> plan;
+  if (best_hg > 0 && best < 0.98 * snake) {
+    sc->hg = best_hg;
+    std::vector<int> owner;
+    list_schedule(causal_costs(*sc, p.geom.Nq), grid, &owner);
+    plan = std::make_shared<attn::FwdPlan>();
+    std::vector<int> count(static_cast<size_t>(grid) + 1, 0);
+    for (int c : owner) ++count[static_cast<size_t>(c) + 1];
+    plan->start[0] = 0;
+    for (int c = 0; c < grid; ++c)
+      plan->start[c + 1] = static_cast<uint16_t>(plan->start[c] + count[static_cast<size_t>(c) + 1]);
+    std::vector<int> fill(plan->start, plan->start + grid);
+    for (size_t idx = 0; idx < owner.size(); ++idx)
+      plan->item[fill[static_cast<size_t>(owner[idx])]++] = static_cast<uint16_t>(idx);
+  } else {
+    sc->hg = snake_hg;
+  }
+  std::lock_guard<std::mutex> g(g_plan_mu);
+  if (g_plans.size() >= 8) g_plans.erase(g_plans.begin());
+  g_plans.push_back(PlanEntry{key, plan, sc->hg});
+  return plan;
+}
+
+template <int D, int MODE, int FEAT, bool PLAN>
+attn_status launch_fwd_kernel(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                              const CUtensorMap& mo, void* o, float* lse, const Problem& p,
+                              const attn::FwdSched& sched, dim3 grid,
+                              const typename attn::FwdPlanArg<PLAN>::type& plan,
+                              cudaStream_t stream) {
   using Cfg = attn::FwdCfg<D>;
-  auto kern = attn::fwd_kernel<D, MODE, FEAT>;
+  auto kern = attn::fwd_kernel<D, MODE, FEAT, PLAN>;
   static KernelSetup setup;
   int launch_regs = 0;
   const cudaError_t attr_err = prepare_kernel(kern, Cfg::kSmemAlloc, setup, &launch_regs);
@@ -426,6 +560,23 @@ attn_status launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUten
   if (launch_regs != attn::kFwdRegsLaunch)
     return fail(ATTN_ERR_CUDA, "fwd kernel built with %d registers/thread, expected %d",
                 launch_regs, attn::kFwdRegsLaunch);
+  const float scale_log2 = p.scale * 1.4426950408889634f;
+  ProfScope ps(kProfFwd, stream);
+  cudaError_t e = launch_pdl(kern, grid, Cfg::kThreads, Cfg::kSmemAlloc, stream, mq, mk, mv, mo,
+                             static_cast<__nv_bfloat16*>(o), lse, p.Hq, p.Hq / p.Hkv, p.geom,
+                             scale_log2, p.mask.win, p.cap, sched, plan);
+  ps.end();
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return cuda_fail(e, "fwd kernel launch");
+  }
+  return ATTN_OK;
+}
+
+template <int D, int MODE, int FEAT>
+attn_status launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                       const CUtensorMap& mo, void* o, float* lse, const Problem& p,
+                       cudaStream_t stream) {
   // Work items are 256-row query blocks: two 128-row tiles share each K/V
   // tile. When there are fewer blocks than SMs, 128-row blocks (one tile)
   // double their number. The grid is persistent: one CTA per SM, or one per
@@ -436,21 +587,20 @@ attn_status launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUten
   sched.one_tile = pairs < sm_count() ? 1 : 0;
   sched.nmb = sched.one_tile ? (p.geom.Nq + 127) / 128 : (p.geom.Nq + 255) / 256;
   sched.total = static_cast<long long>(sched.BH) * sched.nmb;
-  sched.hg = fwd_head_group(p, sched.nmb,
-                            static_cast<int>(std::min<long long>(sched.total, sm_count())));
+  const int g = static_cast<int>(std::min<long long>(sched.total, sm_count()));
+  sched.hg = fwd_head_group(p, sched.nmb, g);
   if (sched.total > 0x7FFFFFFFLL) return fail(ATTN_ERR_ARG, "problem too large for one launch");
-  dim3 grid(static_cast<unsigned>(std::min<long long>(sched.total, sm_count())));
-  const float scale_log2 = p.scale * 1.4426950408889634f;
-  ProfScope ps(kProfFwd, stream);
-  cudaError_t e = launch_pdl(kern, grid, Cfg::kThreads, Cfg::kSmemAlloc, stream, mq, mk, mv, mo,
-                             static_cast<__nv_bfloat16*>(o), lse, p.Hq, p.Hq / p.Hkv, p.geom,
-                             scale_log2, p.mask.win, p.cap, sched);
-  ps.end();
-  if (e != cudaSuccess) {
-    cudaGetLastError();
-    return cuda_fail(e, "fwd kernel launch");
+  const dim3 grid(static_cast<unsigned>(g));
+  if constexpr (MODE == attn::kMaskCausal && FEAT == 0) {
+    if (sched.total > g && sched.total <= attn::kFwdPlanItems && g <= attn::kFwdPlanCtas) {
+      const std::shared_ptr<const attn::FwdPlan> plan = causal_plan(p, g, &sched);
+      if (plan)
+        return launch_fwd_kernel<D, MODE, FEAT, true>(mq, mk, mv, mo, o, lse, p, sched, grid,
+                                                      *plan, stream);
+    }
   }
-  return ATTN_OK;
+  return launch_fwd_kernel<D, MODE, FEAT, false>(mq, mk, mv, mo, o, lse, p, sched, grid,
+                                                 attn::FwdNoPlan{0}, stream);
 }
 
 struct BwdArgs {

@@ -92,15 +92,41 @@ static_assert(2 * kFwdRegsSoftmax + kFwdRegsSmall <= 3 * kFwdRegsLaunch, "regist
 // one (batch, query head), rb = 256 (two tiles) or 128 (one tile, when two-tile
 // blocks would leave SMs idle). Heads are taken in groups of `hg` (see the
 // host), blocks from the last (heaviest when causal) to the first within a
-// group, all heads of the group per block. CTA c of G takes list entries
-// t G + c for even t and t G + G - 1 - c for odd t (a snake), which evens out
-// the work of the CTAs over the heavy-to-light order.
+// group, all heads of the group per block. Without a plan (below), CTA c of
+// G takes list entries t G + c for even t and t G + G - 1 - c for odd t (a
+// snake), which evens out the work of the CTAs over the heavy-to-light order
+// when the blocks cost the same or the list is a whole number of snake periods.
 struct FwdSched {
   int BH;            // batch * query heads
   int nmb;           // query blocks per head (of the longest sequence)
   int hg;            // heads per group
   int one_tile;      // 1: blocks of 128 rows (tile 1 never used)
   long long total;   // BH * nmb (the host keeps it below 2^31)
+};
+
+// A static plan of which CTA takes which list entries, for problems whose
+// blocks differ in cost (causal). CTA c takes entries item[start[c]] ..
+// item[start[c + 1] - 1] in that order. The host fills it by list
+// scheduling: entries in list order, each to the CTA with the least work so
+// far (key-tile steps plus a fixed cost per block). It travels in the kernel
+// parameters, so a launch (or a CUDA graph that captured one) needs no device
+// memory for it.
+constexpr int kFwdPlanCtas = 160;
+constexpr int kFwdPlanItems = 15360;
+struct FwdPlan {
+  uint16_t start[kFwdPlanCtas + 1];
+  uint16_t item[kFwdPlanItems];
+};
+struct FwdNoPlan {
+  int unused;
+};
+template <bool P>
+struct FwdPlanArg {
+  using type = FwdNoPlan;
+};
+template <>
+struct FwdPlanArg<true> {
+  using type = FwdPlan;
 };
 
 struct FwdBlock {
@@ -114,14 +140,23 @@ struct FwdBlock {
 };
 
 // List entry t of this CTA, or false when the list is exhausted.
-template <int MODE, bool PACKED>
-__device__ __forceinline__ bool fwd_block(int t, const FwdSched& sc, int Hq, int group,
-                                          const SeqGeom& geom, KeyWindow win, FwdBlock& bk) {
-  // 32-bit arithmetic: the host keeps the list below 2^31 entries, and
-  // t G + G stays below 2^32 while t G < total.
-  const uint32_t G = gridDim.x, c = blockIdx.x;
-  const uint32_t idx = static_cast<uint32_t>(t) * G + ((t & 1) ? (G - 1 - c) : c);
-  if (idx >= static_cast<uint32_t>(sc.total)) return false;
+template <int MODE, bool PACKED, bool PLAN>
+__device__ __forceinline__ bool fwd_block(int t, const FwdSched& sc,
+                                          const typename FwdPlanArg<PLAN>::type& plan, int Hq,
+                                          int group, const SeqGeom& geom, KeyWindow win,
+                                          FwdBlock& bk) {
+  uint32_t idx;
+  if constexpr (PLAN) {
+    const int s0 = plan.start[blockIdx.x];
+    if (t >= plan.start[blockIdx.x + 1] - s0) return false;
+    idx = plan.item[s0 + t];
+  } else {
+    // 32-bit arithmetic: the host keeps the list below 2^31 entries, and
+    // t G + G stays below 2^32 while t G < total.
+    const uint32_t G = gridDim.x, c = blockIdx.x;
+    idx = static_cast<uint32_t>(t) * G + ((t & 1) ? (G - 1 - c) : c);
+    if (idx >= static_cast<uint32_t>(sc.total)) return false;
+  }
   const uint32_t per_group = static_cast<uint32_t>(sc.hg) * static_cast<uint32_t>(sc.nmb);
   const uint32_t g = idx / per_group;
   const uint32_t r = idx - g * per_group;
@@ -157,13 +192,14 @@ __device__ __forceinline__ bool fwd_block(int t, const FwdSched& sc, int Hq, int
   return true;
 }
 
-template <int D, int MODE, int FEAT>
+template <int D, int MODE, int FEAT, bool PLAN>
 __global__ void __launch_bounds__(384, 1)
 fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
            const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
            __nv_bfloat16* __restrict__ out,
            float* __restrict__ lse_out, int Hq, int group, SeqGeom geom, float scale_log2,
-           KeyWindow win, Softcap cap, FwdSched sched) {
+           KeyWindow win, Softcap cap, FwdSched sched,
+           const __grid_constant__ typename FwdPlanArg<PLAN>::type plan) {
   constexpr bool SOFTCAP = (FEAT & kFeatSoftcap) != 0;
   constexpr bool PACKED = (FEAT & kFeatPacked) != 0;
   static_assert(FEAT == 0 || MODE == kMaskGeneral, "features run in the general mode");
@@ -233,7 +269,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
       int last_q0 = -1, last_q1 = -1;   // block index of the last Q load per set
       bool ok = true;
       FwdBlock bk;
-      for (int t = 0; ok && fwd_block<MODE, PACKED>(t, sched, Hq, group, geom, win, bk); ++t) {
+      for (int t = 0; ok && fwd_block<MODE, PACKED, PLAN>(t, sched, plan, Hq, group, geom, win, bk); ++t) {
         if (!bk.present) continue;
         const int set = k & 1;
         if (k >= 2 && !mbar_wait(&q_empty[set], ((k >> 1) - 1) & 1, abort_flag, kSiteQEmpty)) {
@@ -309,7 +345,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
       uint32_t pc0 = 0, pc1 = 0;
       int oc0 = 0, oc1 = 0;
       FwdBlock bk;
-      for (int t = 0; ok && fwd_block<MODE, PACKED>(t, sched, Hq, group, geom, win, bk); ++t) {
+      for (int t = 0; ok && fwd_block<MODE, PACKED, PLAN>(t, sched, plan, Hq, group, geom, win, bk); ++t) {
         if (!bk.present) continue;
         const int set = k & 1;
         if (!mbar_wait(&q_full[set], (k >> 1) & 1, abort_flag, kSiteQFull)) { ok = false; break; }
@@ -401,7 +437,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
       tma_prefetch_desc(&tm_o);
       int k = 0;
       FwdBlock bk;
-      for (int t = 0; fwd_block<MODE, PACKED>(t, sched, Hq, group, geom, win, bk); ++t) {
+      for (int t = 0; fwd_block<MODE, PACKED, PLAN>(t, sched, plan, Hq, group, geom, win, bk); ++t) {
         if (!bk.present) continue;
         const int set = k & 1;
         bool ok = true;
@@ -443,7 +479,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
     int k = 0;                // present blocks
     bool ok = true;
     FwdBlock bk;
-    for (int it = 0; fwd_block<MODE, PACKED>(it, sched, Hq, group, geom, win, bk); ++it) {
+    for (int it = 0; fwd_block<MODE, PACKED, PLAN>(it, sched, plan, Hq, group, geom, win, bk); ++it) {
       if (!bk.present) continue;
       const int set = k & 1;
       ++k;
