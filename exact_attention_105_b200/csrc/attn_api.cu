@@ -390,6 +390,7 @@ struct Problem {
 //   An L2-sized group that broke the periods was slower (c3 1012 -> 913); the
 //   aligned one is faster (c3 1021 -> 1044, c5 851 -> 861 TFLOP/s).
 // - Other masks (windows): one group.
+// A causal problem that runs with a plan (below) uses the plan's group size.
 int fwd_head_group(const Problem& p, int nmb, int grid) {
   const long long all = static_cast<long long>(p.B) * p.Hq;
   if (p.mask.mode == attn::kMaskCausal) {
