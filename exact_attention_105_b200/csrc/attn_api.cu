@@ -544,14 +544,14 @@ std::shared_ptr<const attn::FwdPlan> causal_plan(const Problem& p, int grid, att
   return plan;
 }
 
-template <int D, int MODE, int FEAT, bool PLAN>
+template <int D, int MODE, int FEAT, bool PLAN, bool DB>
 attn_status launch_fwd_kernel(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                               const CUtensorMap& mo, void* o, float* lse, const Problem& p,
                               const attn::FwdSched& sched, dim3 grid,
                               const typename attn::FwdPlanArg<PLAN>::type& plan,
                               cudaStream_t stream) {
   using Cfg = attn::FwdCfg<D>;
-  auto kern = attn::fwd_kernel<D, MODE, FEAT, PLAN>;
+  auto kern = attn::fwd_kernel<D, MODE, FEAT, PLAN, DB>;
   static KernelSetup setup;
   int launch_regs = 0;
   const cudaError_t attr_err = prepare_kernel(kern, Cfg::kSmemAlloc, setup, &launch_regs);
@@ -592,16 +592,23 @@ attn_status launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUten
   sched.hg = fwd_head_group(p, sched.nmb, g);
   if (sched.total > 0x7FFFFFFFLL) return fail(ATTN_ERR_ARG, "problem too large for one launch");
   const dim3 grid(static_cast<unsigned>(g));
+  // One-tile blocks at d = 64 double-buffer S in the second tile's tensor
+  // memory (there is room: 2 x 128 S columns + 64 O columns).
+  if constexpr (D == 64) {
+    if (sched.one_tile)
+      return launch_fwd_kernel<D, MODE, FEAT, false, true>(mq, mk, mv, mo, o, lse, p, sched, grid,
+                                                           attn::FwdNoPlan{0}, stream);
+  }
   if constexpr (MODE == attn::kMaskCausal && FEAT == 0) {
     if (sched.total > g && sched.total <= attn::kFwdPlanItems && g <= attn::kFwdPlanCtas) {
       const std::shared_ptr<const attn::FwdPlan> plan = causal_plan(p, g, &sched);
       if (plan)
-        return launch_fwd_kernel<D, MODE, FEAT, true>(mq, mk, mv, mo, o, lse, p, sched, grid,
-                                                      *plan, stream);
+        return launch_fwd_kernel<D, MODE, FEAT, true, false>(mq, mk, mv, mo, o, lse, p, sched,
+                                                             grid, *plan, stream);
     }
   }
-  return launch_fwd_kernel<D, MODE, FEAT, false>(mq, mk, mv, mo, o, lse, p, sched, grid,
-                                                 attn::FwdNoPlan{0}, stream);
+  return launch_fwd_kernel<D, MODE, FEAT, false, false>(mq, mk, mv, mo, o, lse, p, sched, grid,
+                                                        attn::FwdNoPlan{0}, stream);
 }
 
 struct BwdArgs {

@@ -35,6 +35,11 @@
 // the tensor pipe executes one thread's MMAs in issue order. The first PV of
 // a block overwrites O_t only after that tile's epilogue of the previous
 // block has read it (o_empty).
+// One-tile blocks at d = 64 (problems too small to fill the SMs with two-tile
+// blocks) run a double-buffered variant: S(j) of the one tile alternates
+// between columns [0, 128) and [128, 256), and S(j + 2) is issued right after
+// PV(j), so the softmax never waits for its own PV and next S. Its O rescale
+// then first waits for PV(j - 1) (pv_done).
 //
 // Shared memory: two sets of Q tiles (the block being computed and the next
 // one), then a ring of NS K/V slots. K_j and V_j take turns: K0, V0, K1, V1,
@@ -62,8 +67,8 @@ struct FwdCfg {
   static constexpr int kKVOff = 4 * kTileBytes;
   static constexpr int kBarOff = kKVOff + kStages * kTileBytes;
   // q_full[2] q_empty[2] kv_full[S] kv_empty[S] s_full[2] p_full[2] p_half[2]
-  // o_full[2] o_empty[2] stage_full[4] mma_done[1]
-  static constexpr int kNumBars = 2 + 2 + 2 * kStages + 2 + 2 + 2 + 2 + 2 + 4 + 1;
+  // o_full[2] o_empty[2] stage_full[4] mma_done[1] pv_done[1]
+  static constexpr int kNumBars = 2 + 2 + 2 * kStages + 2 + 2 + 2 + 2 + 2 + 4 + 1 + 1;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
   static constexpr int kBytes = kMiscOff + 16;
   static constexpr int kSmemAlloc = kBytes + 1024;         // slack for 1024-B alignment
@@ -75,7 +80,8 @@ struct FwdCfg {
 // Wait-site ids reported in the status word when a wait times out.
 enum FwdSite : int {
   kSiteQFull = 1, kSiteKVFull = 2, kSiteKVEmpty = 3, kSiteSFull = 4, kSitePFull = 5,
-  kSiteOFull = 6, kSiteQEmpty = 7, kSiteOEmpty = 8, kSiteStage = 9, kSitePHalf = 10
+  kSiteOFull = 6, kSiteQEmpty = 7, kSiteOEmpty = 8, kSiteStage = 9, kSitePHalf = 10,
+  kSitePVDone = 11
 };
 
 // Register split: launched at kFwdRegsLaunch per thread (384 threads fill the
@@ -192,7 +198,7 @@ __device__ __forceinline__ bool fwd_block(int t, const FwdSched& sc,
   return true;
 }
 
-template <int D, int MODE, int FEAT, bool PLAN>
+template <int D, int MODE, int FEAT, bool PLAN, bool DB>
 __global__ void __launch_bounds__(384, 1)
 fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
            const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
@@ -203,6 +209,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
   constexpr bool SOFTCAP = (FEAT & kFeatSoftcap) != 0;
   constexpr bool PACKED = (FEAT & kFeatPacked) != 0;
   static_assert(FEAT == 0 || MODE == kMaskGeneral, "features run in the general mode");
+  static_assert(!DB || (D == 64 && !PLAN), "double-buffered S: one-tile blocks at d = 64");
   using C = FwdCfg<D>;
   constexpr int NS = C::kStages;
   extern __shared__ uint8_t smem_raw[];
@@ -221,6 +228,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
   uint64_t* o_empty = o_full + 2;         // per tile: the epilogue has read O
   uint64_t* stage_full = o_empty + 2;     // per (Q set, tile): O staged or written directly
   uint64_t* mma_done = stage_full + 4;
+  uint64_t* pv_done = mma_done + 1;       // double-buffered mode: a block's PV (not its last) done
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kMiscOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kMiscOff + 4);
 
@@ -243,6 +251,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
       mbar_init(&kv_empty[i], 1);
     }
     mbar_init(mma_done, 1);
+    mbar_init(pv_done, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -345,87 +354,168 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
       uint32_t pc0 = 0, pc1 = 0;
       int oc0 = 0, oc1 = 0;
       FwdBlock bk;
-      for (int t = 0; ok && fwd_block<MODE, PACKED, PLAN>(t, sched, plan, Hq, group, geom, win, bk); ++t) {
-        if (!bk.present) continue;
-        const int set = k & 1;
-        if (!mbar_wait(&q_full[set], (k >> 1) & 1, abort_flag, kSiteQFull)) { ok = false; break; }
-        ++k;
-        if (bk.n_span == 0) continue;
-        any = true;
-        const int jb = bk.jb, je = bk.jb + bk.n_span;
-        auto lo_t = [&](int tt) { return tt ? bk.lo1 : bk.lo0; };
-        auto hi_t = [&](int tt) { return tt ? bk.hi1 : bk.hi0; };
-        // Ring positions: K_j at base + 2 (j - jb), V_j at base + 2 (j - jb) + 1.
-        if (!kv_wait(base)) { ok = false; break; }
-        tc_fence_after();
+      if constexpr (DB) {
+        // One-tile blocks with S double-buffered in TMEM columns [0, 128) and
+        // [128, 256) (the second tile's, unused here): S(j + 2) is issued right
+        // after PV(j), so the softmax finds S(j + 1) ready when it finishes
+        // S(j) instead of waiting for PV(j) and S(j + 1) in turn.
+        auto issue_qk_db = [&](uint32_t b, int set, uint32_t slot) {
+          const SDesc qd =
+              sdesc_sw128_split(sbase + C::kQOff + 2 * set * C::kTileBytes, 16, 1024);
+          const SDesc kd = sdesc_sw128_split(sbase + C::kKVOff + slot * C::kTileBytes, 16, 1024);
+          mma_ss_w<0>(tmem + b * 128, qd.lo, qd.hi, kd.lo, kd.hi, kIdescQK);
 #pragma unroll
-        for (int tt = 0; tt < 2; ++tt)
-          if (hi_t(tt) >= lo_t(tt) && lo_t(tt) == jb) {
-            issue_qk(tt, set, base % NS);
-            tc_commit(&s_full[tt]);
+          for (int kk = 1; kk < D / 16; ++kk) {
+            const uint32_t o = ((kk >> 2) * 16384 + (kk & 3) * 32) >> 4;
+            mma_ss_w<1>(tmem + b * 128, qd.lo + o, qd.hi, kd.lo + o, kd.hi, kIdescQK);
           }
-        tc_commit(&kv_empty[base % NS]);
-        for (int j = jb; ok && j < je; ++j) {
-          const uint32_t iv = base + 2 * (j - jb) + 1, ik = iv + 1;
-          if (!kv_wait(iv)) { ok = false; break; }
-          tc_fence_after();
-          bool k_ready = false;
-          auto need_k_next = [&]() {
-            if (!k_ready) {
-              if (!kv_wait(ik)) return false;
-              tc_fence_after();
-              k_ready = true;
-            }
-            return true;
-          };
+        };
+        auto issue_pv_db = [&](uint32_t b, uint32_t slot, int h, bool acc) {
+          const SDesc vd =
+              sdesc_sw128_split(sbase + C::kKVOff + slot * C::kTileBytes, 16384, 1024);
+          const uint32_t pa = tmem + b * 128 + 64 + 32 * h, od = tmem + 256;
+          mma_ts_w<-1>(od, pa, vd.lo + 4 * h * 128, vd.hi, kIdescPV, acc ? 1u : 0u);
 #pragma unroll
-          for (int tt = 0; tt < 2; ++tt) {
-            const int lo = lo_t(tt), hi = hi_t(tt);
-            if (hi < lo) continue;
-            if (j >= lo && j <= hi) {
-              uint32_t& pc = tt ? pc1 : pc0;
-              int& oc = tt ? oc1 : oc0;
-              // P arrives in two halves: the first half's PV runs while the
-              // softmax still computes the second half. The next S tile
-              // overwrites P, so it follows the second half's PV.
-              if (!mbar_wait(&p_half[tt], pc & 1u, abort_flag, kSitePHalf)) { ok = false; break; }
-              // The first accumulation of a block overwrites O_t: the previous
-              // block's epilogue must have read it.
-              if (j == lo && oc > 0 &&
-                  !mbar_wait(&o_empty[tt], (oc - 1) & 1, abort_flag, kSiteOEmpty)) {
-                ok = false;
-                break;
+          for (int kk = 1; kk < 4; ++kk)
+            mma_ts_w<1>(od, pa + kk * 8, vd.lo + (4 * h + kk) * 128, vd.hi, kIdescPV);
+        };
+        for (int t = 0; ok && fwd_block<MODE, PACKED, PLAN>(t, sched, plan, Hq, group, geom, win, bk);
+             ++t) {
+          if (!bk.present) continue;
+          const int set = k & 1;
+          if (!mbar_wait(&q_full[set], (k >> 1) & 1, abort_flag, kSiteQFull)) { ok = false; break; }
+          ++k;
+          const int n = bk.n_span;        // the one tile's key tiles are the block's span
+          if (n == 0) continue;
+          any = true;
+          // K of the block's key tile jj at base + 2 jj, its V at base + 2 jj + 1.
+          for (int jj = 0; ok && jj < 2 && jj < n; ++jj) {
+            if (!kv_wait(base + 2 * jj)) { ok = false; break; }
+            tc_fence_after();
+            issue_qk_db(jj, set, (base + 2 * jj) % NS);
+            tc_commit(&s_full[jj]);
+            tc_commit(&kv_empty[(base + 2 * jj) % NS]);
+          }
+          for (int jj = 0; ok && jj < n; ++jj) {
+            const uint32_t b = jj & 1, iv = base + 2 * jj + 1;
+            if (!kv_wait(iv) || !mbar_wait(&p_half[0], pc0 & 1u, abort_flag, kSitePHalf)) {
+              ok = false;
+              break;
+            }
+            if (jj == 0 && oc0 > 0 &&
+                !mbar_wait(&o_empty[0], (oc0 - 1) & 1, abort_flag, kSiteOEmpty)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            issue_pv_db(b, iv % NS, 0, jj > 0);
+            if (!mbar_wait(&p_full[0], pc0 & 1u, abort_flag, kSitePFull)) { ok = false; break; }
+            ++pc0;
+            tc_fence_after();
+            issue_pv_db(b, iv % NS, 1, true);
+            if (jj == n - 1) {
+              tc_commit(&o_full[0]);
+              ++oc0;
+            } else {
+              tc_commit(pv_done);
+            }
+            tc_commit(&kv_empty[iv % NS]);
+            if (jj + 2 < n) {
+              // Into the buffer PV(jj) has just read: the pipe runs this
+              // thread's MMAs in issue order.
+              const uint32_t ik = base + 2 * (jj + 2);
+              if (!kv_wait(ik)) { ok = false; break; }
+              tc_fence_after();
+              issue_qk_db(b, set, ik % NS);
+              tc_commit(&s_full[b]);
+              tc_commit(&kv_empty[ik % NS]);
+            }
+          }
+          base += 2 * n;
+        }
+      } else {
+        for (int t = 0; ok && fwd_block<MODE, PACKED, PLAN>(t, sched, plan, Hq, group, geom, win, bk); ++t) {
+          if (!bk.present) continue;
+          const int set = k & 1;
+          if (!mbar_wait(&q_full[set], (k >> 1) & 1, abort_flag, kSiteQFull)) { ok = false; break; }
+          ++k;
+          if (bk.n_span == 0) continue;
+          any = true;
+          const int jb = bk.jb, je = bk.jb + bk.n_span;
+          auto lo_t = [&](int tt) { return tt ? bk.lo1 : bk.lo0; };
+          auto hi_t = [&](int tt) { return tt ? bk.hi1 : bk.hi0; };
+          // Ring positions: K_j at base + 2 (j - jb), V_j at base + 2 (j - jb) + 1.
+          if (!kv_wait(base)) { ok = false; break; }
+          tc_fence_after();
+  #pragma unroll
+          for (int tt = 0; tt < 2; ++tt)
+            if (hi_t(tt) >= lo_t(tt) && lo_t(tt) == jb) {
+              issue_qk(tt, set, base % NS);
+              tc_commit(&s_full[tt]);
+            }
+          tc_commit(&kv_empty[base % NS]);
+          for (int j = jb; ok && j < je; ++j) {
+            const uint32_t iv = base + 2 * (j - jb) + 1, ik = iv + 1;
+            if (!kv_wait(iv)) { ok = false; break; }
+            tc_fence_after();
+            bool k_ready = false;
+            auto need_k_next = [&]() {
+              if (!k_ready) {
+                if (!kv_wait(ik)) return false;
+                tc_fence_after();
+                k_ready = true;
               }
-              tc_fence_after();
-              issue_pv_half(tt, iv % NS, 0, j > lo);
-              if (!mbar_wait(&p_full[tt], pc & 1u, abort_flag, kSitePFull)) { ok = false; break; }
-              ++pc;
-              tc_fence_after();
-              issue_pv_half(tt, iv % NS, 1, true);
-              if (j == hi) {
-                tc_commit(&o_full[tt]);
-                ++oc;
-              } else {
+              return true;
+            };
+  #pragma unroll
+            for (int tt = 0; tt < 2; ++tt) {
+              const int lo = lo_t(tt), hi = hi_t(tt);
+              if (hi < lo) continue;
+              if (j >= lo && j <= hi) {
+                uint32_t& pc = tt ? pc1 : pc0;
+                int& oc = tt ? oc1 : oc0;
+                // P arrives in two halves: the first half's PV runs while the
+                // softmax still computes the second half. The next S tile
+                // overwrites P, so it follows the second half's PV.
+                if (!mbar_wait(&p_half[tt], pc & 1u, abort_flag, kSitePHalf)) { ok = false; break; }
+                // The first accumulation of a block overwrites O_t: the previous
+                // block's epilogue must have read it.
+                if (j == lo && oc > 0 &&
+                    !mbar_wait(&o_empty[tt], (oc - 1) & 1, abort_flag, kSiteOEmpty)) {
+                  ok = false;
+                  break;
+                }
+                tc_fence_after();
+                issue_pv_half(tt, iv % NS, 0, j > lo);
+                if (!mbar_wait(&p_full[tt], pc & 1u, abort_flag, kSitePFull)) { ok = false; break; }
+                ++pc;
+                tc_fence_after();
+                issue_pv_half(tt, iv % NS, 1, true);
+                if (j == hi) {
+                  tc_commit(&o_full[tt]);
+                  ++oc;
+                } else {
+                  if (!need_k_next()) { ok = false; break; }
+                  issue_qk(tt, set, ik % NS);
+                  tc_commit(&s_full[tt]);
+                }
+              } else if (lo == j + 1) {
+                // This tile's first key tile is the next one.
                 if (!need_k_next()) { ok = false; break; }
                 issue_qk(tt, set, ik % NS);
                 tc_commit(&s_full[tt]);
               }
-            } else if (lo == j + 1) {
-              // This tile's first key tile is the next one.
-              if (!need_k_next()) { ok = false; break; }
-              issue_qk(tt, set, ik % NS);
-              tc_commit(&s_full[tt]);
             }
+            // K_{j+1} feeds some tile whenever j + 1 is in the span (the two
+            // tiles' ranges overlap or touch); release its slot even if no tile
+            // used it.
+            if (ok && j + 1 < je && !need_k_next()) ok = false;
+            if (!ok) break;
+            tc_commit(&kv_empty[iv % NS]);
+            if (k_ready) tc_commit(&kv_empty[ik % NS]);
           }
-          // K_{j+1} feeds some tile whenever j + 1 is in the span (the two
-          // tiles' ranges overlap or touch); release its slot even if no tile
-          // used it.
-          if (ok && j + 1 < je && !need_k_next()) ok = false;
-          if (!ok) break;
-          tc_commit(&kv_empty[iv % NS]);
-          if (k_ready) tc_commit(&kv_empty[ik % NS]);
+          base += 2 * bk.n_span;
         }
-        base += 2 * bk.n_span;
       }
       // Let this thread's MMAs finish before TMEM can be released.
       if (any) {
@@ -475,6 +565,8 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
     const uint32_t t_o = tmem + lane_base + 256 + t * 128;
     const int tr = quad * 32 + lane;                       // row within the tile
     uint32_t sc = 0;          // S hand-overs consumed by this tile
+    uint32_t sc1 = 0;         // double-buffered mode: those of the second buffer
+    uint32_t pvc = 0;         // double-buffered mode: PV completions waited for
     int oc = 0;               // blocks whose O this tile accumulated
     int k = 0;                // present blocks
     bool ok = true;
@@ -514,14 +606,20 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
       for (int jj = 0; ok && jj < n; ++jj) {
         const int j = lo + jj;                             // key tile
         const int kb = j * 128;
-        if (!mbar_wait(&s_full[t], sc & 1u, abort_flag, kSiteSFull)) { ok = false; break; }
-        ++sc;
+        // Double-buffered mode: odd steps use the second S buffer and barrier.
+        const bool odd = DB && (jj & 1);
+        const uint32_t t_sb = odd ? t_s + 128 : t_s;
+        if (!mbar_wait(&s_full[odd ? 1 : t], (odd ? sc1 : sc) & 1u, abort_flag, kSiteSFull)) {
+          ok = false;
+          break;
+        }
+        if (odd) ++sc1; else ++sc;
         tc_fence_after();
         uint32_t r0[32], r1[32], r2[32], r3[32];
-        tmem_ld32(t_s + 0, r0);
-        tmem_ld32(t_s + 32, r1);
-        tmem_ld32(t_s + 64, r2);
-        tmem_ld32(t_s + 96, r3);
+        tmem_ld32(t_sb + 0, r0);
+        tmem_ld32(t_sb + 32, r1);
+        tmem_ld32(t_sb + 64, r2);
+        tmem_ld32(t_sb + 96, r3);
         tmem_ld_wait(r0);
         reg_fence(r1);
         reg_fence(r2);
@@ -579,6 +677,14 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
         const float m_new = fmaxf(m_run, m_tile);
         // Lazy rescale: keep the stale max unless the new one is more than 2^8 larger.
         const bool need = m_new > m_run + 8.0f;
+        if constexpr (DB) {
+          // S(jj) was issued before PV(jj - 1), which may still be adding to O.
+          if (jj > 0) {
+            if (!mbar_wait(pv_done, pvc & 1u, abort_flag, kSitePVDone)) { ok = false; break; }
+            ++pvc;
+            tc_fence_after();
+          }
+        }
         if (jj > 0 && __any_sync(0xffffffffu, need)) {
           const float f = need ? fast_exp2(m_run - m_new) : 1.0f;
 #pragma unroll
@@ -637,13 +743,13 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
         // handed over first; keys 64..127 go to columns 96..127.
         emit(r0, 0);
         emit(r1, 16);
-        tmem_st32(t_s + 64, *reinterpret_cast<const uint32_t(*)[32]>(pall));
+        tmem_st32(t_sb + 64, *reinterpret_cast<const uint32_t(*)[32]>(pall));
         emit(r2, 32);
         tmem_st_wait();
         tc_fence_before();
         mbar_arrive(&p_half[t]);
         emit(r3, 48);
-        tmem_st32(t_s + 96, *reinterpret_cast<const uint32_t(*)[32]>(pall + 32));
+        tmem_st32(t_sb + 96, *reinterpret_cast<const uint32_t(*)[32]>(pall + 32));
         const float2 ex = fadd2(ex0, ex1);
         l_run += ex.x + ex.y;
         l_mma += (q0 + q1) + (q2 + q3);
