@@ -592,13 +592,11 @@ attn_status launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUten
   sched.hg = fwd_head_group(p, sched.nmb, g);
   if (sched.total > 0x7FFFFFFFLL) return fail(ATTN_ERR_ARG, "problem too large for one launch");
   const dim3 grid(static_cast<unsigned>(g));
-  // One-tile blocks at d = 64 double-buffer S in the second tile's tensor
-  // memory (there is room: 2 x 128 S columns + 64 O columns).
-  if constexpr (D == 64) {
-    if (sched.one_tile)
-      return launch_fwd_kernel<D, MODE, FEAT, false, true>(mq, mk, mv, mo, o, lse, p, sched, grid,
-                                                           attn::FwdNoPlan{0}, stream);
-  }
+  // One-tile blocks double-buffer S in the second tile's tensor memory
+  // (2 x 128 S columns + D O columns).
+  if (sched.one_tile)
+    return launch_fwd_kernel<D, MODE, FEAT, false, true>(mq, mk, mv, mo, o, lse, p, sched, grid,
+                                                         attn::FwdNoPlan{0}, stream);
   if constexpr (MODE == attn::kMaskCausal && FEAT == 0) {
     if (sched.total > g && sched.total <= attn::kFwdPlanItems && g <= attn::kFwdPlanCtas) {
       const std::shared_ptr<const attn::FwdPlan> plan = causal_plan(p, g, &sched);

@@ -35,11 +35,12 @@
 // the tensor pipe executes one thread's MMAs in issue order. The first PV of
 // a block overwrites O_t only after that tile's epilogue of the previous
 // block has read it (o_empty).
-// One-tile blocks at d = 64 (problems too small to fill the SMs with two-tile
-// blocks) run a double-buffered variant: S(j) of the one tile alternates
-// between columns [0, 128) and [128, 256), and S(j + 2) is issued right after
-// PV(j), so the softmax never waits for its own PV and next S. Its O rescale
-// then first waits for PV(j - 1) (pv_done).
+// One-tile blocks (problems too small to fill the SMs with two-tile blocks)
+// run a double-buffered variant: S(j) of the one tile alternates between
+// columns [0, 128) and [128, 256), and S(j + 2) is issued right after PV(j),
+// so the softmax never waits for its own PV and next S. Its O rescale then
+// first waits for PV(j - 1) (pv_done). The producer loads each K one key tile
+// ahead of its V, so that with a 3-slot ring K(j + 2) is in place by then.
 //
 // Shared memory: two sets of Q tiles (the block being computed and the next
 // one), then a ring of NS K/V slots. K_j and V_j take turns: K0, V0, K1, V1,
@@ -209,7 +210,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
   constexpr bool SOFTCAP = (FEAT & kFeatSoftcap) != 0;
   constexpr bool PACKED = (FEAT & kFeatPacked) != 0;
   static_assert(FEAT == 0 || MODE == kMaskGeneral, "features run in the general mode");
-  static_assert(!DB || (D == 64 && !PLAN), "double-buffered S: one-tile blocks at d = 64");
+  static_assert(!DB || !PLAN, "double-buffered S: one-tile blocks, no plan");
   using C = FwdCfg<D>;
   constexpr int NS = C::kStages;
   extern __shared__ uint8_t smem_raw[];
@@ -294,20 +295,51 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
                         &q_full[set], a * 64, bk.sp.q0 + bk.m0 + tt * 128, bk.zq);
         }
         if (set) last_q1 = k; else last_q0 = k;
-        for (int j = bk.jb; ok && j < bk.jb + bk.n_span; ++j) {
-          for (int w = 0; w < 2; ++w) {
+        if constexpr (DB) {
+          // Next ring load: K (w = 0) or V (w = 1) of key tile j.
+          auto load = [&](int w, int j) {
             const uint32_t s = ld % NS;
             if (ld >= static_cast<uint32_t>(NS) &&
-                !mbar_wait(&kv_empty[s], (ld / NS - 1) & 1u, abort_flag, kSiteKVEmpty)) {
-              ok = false;
-              break;
-            }
+                !mbar_wait(&kv_empty[s], (ld / NS - 1) & 1u, abort_flag, kSiteKVEmpty))
+              return false;
             mbar_expect_tx(&kv_full[s], C::kTxBytes);
 #pragma unroll
             for (int a = 0; a < D / 64; ++a)
               tma_load_3d(smem + C::kKVOff + s * C::kTileBytes + a * 16384, w ? &tm_v : &tm_k,
                           &kv_full[s], a * 64, bk.sp.k0 + j * 128, bk.zkv);
             ++ld;
+            return true;
+          };
+          // With a 3-slot ring, K runs one key tile ahead: K_0, then K_m,
+          // V_(m-1) for m = 1 .. n-1, then V_(n-1), so that K_(j+2) can land
+          // during the softmax of S(j). Deeper rings keep the plain order
+          // (measured 3 % faster at d = 64).
+          const int n = bk.n_span;
+          if (NS < 4) {
+            for (int m = 0; ok && m <= n; ++m) {
+              if (m < n && !load(0, bk.jb + m)) ok = false;
+              if (ok && m > 0 && !load(1, bk.jb + m - 1)) ok = false;
+            }
+          } else {
+            for (int m = 0; ok && m < n; ++m)
+              if (!load(0, bk.jb + m) || !load(1, bk.jb + m)) ok = false;
+          }
+        } else {
+          for (int j = bk.jb; ok && j < bk.jb + bk.n_span; ++j) {
+            for (int w = 0; w < 2; ++w) {
+              const uint32_t s = ld % NS;
+              if (ld >= static_cast<uint32_t>(NS) &&
+                  !mbar_wait(&kv_empty[s], (ld / NS - 1) & 1u, abort_flag, kSiteKVEmpty)) {
+                ok = false;
+                break;
+              }
+              mbar_expect_tx(&kv_full[s], C::kTxBytes);
+#pragma unroll
+              for (int a = 0; a < D / 64; ++a)
+                tma_load_3d(smem + C::kKVOff + s * C::kTileBytes + a * 16384, w ? &tm_v : &tm_k,
+                            &kv_full[s], a * 64, bk.sp.k0 + j * 128, bk.zkv);
+              ++ld;
+            }
           }
         }
         ++k;
@@ -388,16 +420,25 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
           const int n = bk.n_span;        // the one tile's key tiles are the block's span
           if (n == 0) continue;
           any = true;
-          // K of the block's key tile jj at base + 2 jj, its V at base + 2 jj + 1.
+          // Ring positions in the producer's order, from the block's first
+          // load. 3-slot ring (K one key tile ahead): K_m at 2m - 1 (K_0 at
+          // 0), V_m at 2m + 2 (the last V at 2n - 1). Deeper rings: K_m at
+          // 2m, V_m at 2m + 1.
+          auto pos_k = [&](int m) {
+            return base + (NS >= 4 ? 2u * m : (m == 0 ? 0u : 2u * m - 1u));
+          };
+          auto pos_v = [&](int m) {
+            return base + (NS >= 4 ? 2u * m + 1u : (m == n - 1 ? 2u * n - 1u : 2u * m + 2u));
+          };
           for (int jj = 0; ok && jj < 2 && jj < n; ++jj) {
-            if (!kv_wait(base + 2 * jj)) { ok = false; break; }
+            if (!kv_wait(pos_k(jj))) { ok = false; break; }
             tc_fence_after();
-            issue_qk_db(jj, set, (base + 2 * jj) % NS);
+            issue_qk_db(jj, set, pos_k(jj) % NS);
             tc_commit(&s_full[jj]);
-            tc_commit(&kv_empty[(base + 2 * jj) % NS]);
+            tc_commit(&kv_empty[pos_k(jj) % NS]);
           }
           for (int jj = 0; ok && jj < n; ++jj) {
-            const uint32_t b = jj & 1, iv = base + 2 * jj + 1;
+            const uint32_t b = jj & 1, iv = pos_v(jj);
             if (!kv_wait(iv) || !mbar_wait(&p_half[0], pc0 & 1u, abort_flag, kSitePHalf)) {
               ok = false;
               break;
@@ -423,7 +464,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
             if (jj + 2 < n) {
               // Into the buffer PV(jj) has just read: the pipe runs this
               // thread's MMAs in issue order.
-              const uint32_t ik = base + 2 * (jj + 2);
+              const uint32_t ik = pos_k(jj + 2);
               if (!kv_wait(ik)) { ok = false; break; }
               tc_fence_after();
               issue_qk_db(b, set, ik % NS);
