@@ -31,7 +31,11 @@
  *    be 16-byte aligned and must not alias another argument. The library
  *    allocates no memory and keeps no pointer after a call returns.
  *  - Calls are asynchronous on `stream` (a cudaStream_t, may be 0), like a
- *    kernel launch. They return after the launches are queued.
+ *    kernel launch. They return after the launches are queued. The kernels
+ *    are launched with programmatic stream serialization: one may start its
+ *    set-up while the work before it on the stream finishes, but it touches
+ *    no global memory until that work has completed, so the stream order a
+ *    caller sees is that of ordinary launches.
  *  - Supported: d in {64, 128}; N >= 1 (any length; ragged tail tiles are
  *    masked); B, Hq, Hkv >= 1; Hq % Hkv == 0; scale finite and > 0.
  *    B == 0 or N == 0 is an empty problem: nothing is launched and ATTN_OK
