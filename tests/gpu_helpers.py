@@ -21,8 +21,12 @@ def to_dev(*ts):
 
 
 def gpu_fwd(q, k, v, scale, causal):
+    """Forward through the binding into outputs pre-filled with NaN, so a
+    finiteness check over the whole output shows every element was written."""
     qd, kd, vd = to_dev(q, k, v)
-    o, lse = ea.attn_fwd(qd, kd, vd, scale=scale, causal=causal)
+    o = torch.full_like(qd, float("nan"))
+    lse = torch.full(qd.shape[:3], float("nan"), dtype=torch.float32, device=qd.device)
+    ea.attn_fwd(qd, kd, vd, o, lse, scale=scale, causal=causal)
     ea.attn_check_status()
     return o, lse
 

@@ -22,9 +22,12 @@ pytestmark = pytest.mark.gpu
 
 
 def gpu_fwd_bwd(q, k, v, do, scale, causal):
+    """Forward and backward into gradients pre-filled with NaN (see
+    assert_grads_close, which checks the whole of each gradient is finite)."""
     qd, kd, vd, dod = to_dev(q, k, v, do)
     o, lse = ea.attn_fwd(qd, kd, vd, scale=scale, causal=causal)
-    dq, dk, dv = ea.attn_bwd(qd, kd, vd, o, lse, dod, scale=scale, causal=causal)
+    dq, dk, dv = (torch.full_like(t, float("nan")) for t in (qd, kd, vd))
+    ea.attn_bwd(qd, kd, vd, o, lse, dod, dq, dk, dv, scale=scale, causal=causal)
     ea.attn_check_status()
     return dq, dk, dv
 
@@ -33,6 +36,7 @@ def assert_grads_close(got, refs, label, heads=None):
     errs = {}
     for name, g, ref in zip(("dq", "dk", "dv"), got, refs):
         g = g.float().cpu().numpy()
+        assert np.all(np.isfinite(g)), f"{label}: non-finite {name} (an element left unwritten?)"
         if heads is not None:
             sel = heads[name]
             g = np.stack([g[b, h] for b, h in sel])
