@@ -117,6 +117,49 @@ def test_fast_and_checked_paths_agree():
         ea.attn_bwd(q, k, v, o2, lse2, do, dq2.float(), dk2, dv2, ws, causal=True)
 
 
+# Causal shapes whose block count makes the host build a block plan (more
+# distinct shapes than the plan cache holds, so entries are evicted while other
+# threads launch with them).
+PLAN_SHAPES = [(3, 16, 1700, 64), (4, 12, 1700, 64), (3, 12, 2300, 64), (2, 20, 2300, 64),
+               (2, 16, 2900, 64), (4, 8, 2900, 64), (3, 16, 1700, 128), (4, 12, 1700, 128),
+               (2, 12, 3500, 64), (3, 8, 3500, 64)]
+
+
+def test_causal_plans_from_several_host_threads():
+    problems = []
+    for i, (B, H, N, d) in enumerate(PLAN_SHAPES):
+        q, k, v, _ = workloads.make_inputs_qk(B, H, H, N, N, d, seed=100 + i)
+        problems.append(tuple(t.cuda() for t in (q, k, v)))
+    refs = [ea.attn_fwd(q, k, v, causal=True) for q, k, v in problems]
+    torch.cuda.synchronize()
+    results, errors = {}, []
+
+    def worker(w):
+        try:
+            s = torch.cuda.Stream()
+            with torch.cuda.stream(s):
+                n = len(problems)
+                order = [(i + 3 * w) % n for i in range(n)]
+                for _ in range(2):
+                    for i in (order[::-1] if w % 2 else order):
+                        results[(w, i)] = ea.attn_fwd(*problems[i], causal=True)
+            s.synchronize()
+        except Exception as e:     # reported below, on the main thread
+            errors.append(repr(e))
+
+    threads = [threading.Thread(target=worker, args=(w,)) for w in range(3)]
+    for th in threads:
+        th.start()
+    for th in threads:
+        th.join()
+    assert not errors, errors
+    torch.cuda.synchronize()
+    ea.attn_check_status()
+    assert results
+    for (w, i), (o, lse) in results.items():
+        assert torch.equal(o, refs[i][0]) and torch.equal(lse, refs[i][1]), (w, PLAN_SHAPES[i])
+
+
 def test_calls_from_several_host_threads():
     problems = [_problem(10 + i, N=300 + 200 * i) for i in range(4)]
     refs = [_eager(*p) for p in problems]
