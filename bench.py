@@ -367,12 +367,14 @@ def variant_targets(ea, torch, peak, iters=5, warmup=2):
     return out
 
 
-def small_target(ea, torch, w, hbm_gbs, iters=50, warmup=5):
+def small_target(ea, torch, w, hbm_gbs, iters=200, warmup=20):
     """The small configurations are latency-bound. Reports microseconds per
     forward and per forward + backward, called through the API from Python
     (host overhead included) and replayed from a CUDA graph that captured the
     same calls (device time only), plus the forward's HBM byte rate (q, k, v
-    read and o, lse written once) from the graph timing."""
+    read and o, lse written once) from the graph timing. Each figure averages
+    200 back-to-back calls: a call costs microseconds, so fewer calls let one
+    host hiccup move the mean by tens of percent."""
     q, k, v, do = (t.cuda() for t in workloads.make_inputs(w, with_grad_out=True))
     o = torch.empty_like(q)
     lse = torch.empty(q.shape[:3], dtype=torch.float32, device="cuda")
