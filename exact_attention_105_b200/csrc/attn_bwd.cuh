@@ -19,7 +19,12 @@
 //                    stay in shared memory. It loops over the 128-query blocks
 //                    of every query head in the GQA group (from the diagonal
 //                    when causal). Per block it computes S^T, dP^T, P^T, dS^T
-//                    and accumulates dV and dK in TMEM.
+//                    and accumulates dV and dK in TMEM: S^T (then P^T) in
+//                    columns [0, 128), dP^T (then dS^T) in [128, 256), dV in
+//                    [256, 256 + d), dK in [384, 512). At d = 64 the free
+//                    columns hold a second S^T buffer ([384, 512), dK moves to
+//                    [320, 384)) for odd steps, so S^T(s+2) is issued right
+//                    after dV(s) and the compute warps find S^T(s+1) ready.
 //   bwd_dq_kernel    one CTA per (batch, query head, 128-query block). Q_i and
 //                    dO_i stay resident while K_j and V_j stream through two
 //                    rings (K_j is held from S(j) to dQ(j), V_j only for dP(j)).
@@ -223,8 +228,12 @@ struct DkdvCfg {
   static constexpr int kStageBytes = 2 * kTile + 1024;   // Q, dO, 128 L floats, 128 D floats
   static constexpr int kBarOff = kStageOff + kStages * kStageBytes;
   // kv_full kv_empty ld_full[S] ld_empty[S] s_full dp_full p_full ds_full acc_full
-  // stage_full item_full[I] item_empty[I] mma_done
-  static constexpr int kNumBars = 2 + 2 * kStages + 6 + 2 * kItemSlots + 1;
+  // stage_full item_full[I] item_empty[I] mma_done s_full2
+  static constexpr int kNumBars = 2 + 2 * kStages + 6 + 2 * kItemSlots + 1 + 1;
+  // d = 64 leaves 128 tensor-memory columns free: S^T is double-buffered
+  // there (columns [384, 512)), with dK moved to [320, 384).
+  static constexpr bool kDB = D == 64;
+  static constexpr int kDkCol = kDB ? 320 : 384;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
   static constexpr int kBytes = kMiscOff + 8 + 4 * kItemSlots;  // TMEM slot, abort flag, items
   static constexpr int kSmemAlloc = kBytes + 1024;
@@ -302,9 +311,15 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   uint64_t* item_full = stage_full + 1;
   uint64_t* item_empty = item_full + IS;
   uint64_t* mma_done = item_empty + IS;
+  uint64_t* s_full2 = mma_done + 1;       // double-buffered mode: S^T of odd steps
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kMiscOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kMiscOff + 4);
   volatile int* item_slot = reinterpret_cast<volatile int*>(smem + C::kMiscOff + 8);
+  constexpr bool DB = C::kDB;
+  // S^T buffer and its barrier for step g.
+  auto s_col = [&](uint32_t g) { return (DB && (g & 1)) ? 384u : 0u; };
+  auto s_bar = [&](uint32_t g) { return (DB && (g & 1)) ? s_full2 : s_full; };
+  auto s_par = [&](uint32_t g) { return DB ? (g >> 1) & 1u : g & 1u; };
 
   const int warp = warp_id(), lane = lane_id();
   const int Hkv = Hq / group;
@@ -328,6 +343,7 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       mbar_init(&item_empty[s], kItemReaders);
     }
     mbar_init(mma_done, 1);
+    mbar_init(s_full2, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -473,30 +489,43 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         ++kv_loads;
         any = true;
         tc_fence_after();
-        mma_tile_kk(tmem + 0, sbase + C::kKOff, stage_addr(g));                 // S^T(0)
-        tc_commit(s_full);
+        mma_tile_kk(tmem + s_col(g), sbase + C::kKOff, stage_addr(g));          // S^T(0)
+        tc_commit(s_bar(g));
         mma_tile_kk(tmem + 128, sbase + C::kVOff, stage_addr(g) + C::kTile);    // dP^T(0)
         tc_commit(dp_full);
+        if (DB && n > 1) {
+          // S^T(1) into the second buffer right away.
+          if (!mbar_wait(&ld_full[(g + 1) % NS], ((g + 1) / NS) & 1u, abort_flag,
+                         kSiteBLoadFull)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          mma_tile_kk(tmem + s_col(g + 1), sbase + C::kKOff, stage_addr(g + 1));
+          tc_commit(s_bar(g + 1));
+        }
         if (n == 1) tc_commit(kv_empty);
         for (int s = 0; ok && s < n; ++s, ++g) {
           const uint32_t sa = stage_addr(g);
           if (!mbar_wait(p_full, g & 1u, abort_flag, kSiteBP)) { ok = false; break; }
           tc_fence_after();
-          mma_acc(tmem + 256, tmem + 0, sa + C::kTile, s > 0);                    // dV += P^T dO
+          mma_acc(tmem + 256, tmem + s_col(g), sa + C::kTile, s > 0);             // dV += P^T dO
           const bool more = s + 1 < n;
-          if (more) {
-            if (!mbar_wait(&ld_full[(g + 1) % NS], ((g + 1) / NS) & 1u, abort_flag,
-                           kSiteBLoadFull)) {
+          // S^T of a later step: the next one (single buffer, after dV has
+          // read P^T from its columns), or the one after (double-buffered).
+          const uint32_t gn = DB ? g + 2 : g + 1;
+          if (DB ? s + 2 < n : more) {
+            if (!mbar_wait(&ld_full[gn % NS], (gn / NS) & 1u, abort_flag, kSiteBLoadFull)) {
               ok = false;
               break;
             }
             tc_fence_after();
-            mma_tile_kk(tmem + 0, sbase + C::kKOff, stage_addr(g + 1));          // S^T(s+1)
-            tc_commit(s_full);
+            mma_tile_kk(tmem + s_col(gn), sbase + C::kKOff, stage_addr(gn));     // S^T
+            tc_commit(s_bar(gn));
           }
           if (!mbar_wait(ds_full, g & 1u, abort_flag, kSiteBDS)) { ok = false; break; }
           tc_fence_after();
-          mma_acc(tmem + 384, tmem + 128, sa, s > 0);                             // dK += dS^T Q
+          mma_acc(tmem + C::kDkCol, tmem + 128, sa, s > 0);                       // dK += dS^T Q
           if (more) {
             // The last step's stage is released by the store thread instead.
             tc_commit(&ld_empty[g % NS]);
@@ -583,14 +612,15 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                                                          2 * C::kTile) + c_base;
         const float* Ds = Ls + 128;
         if (!mbar_wait(&ld_full[st], (g / NS) & 1u, abort_flag, kSiteBLoadFull) ||
-            !mbar_wait(s_full, g & 1u, abort_flag, kSiteBS)) {
+            !mbar_wait(s_bar(g), s_par(g), abort_flag, kSiteBS)) {
           ok = false;
           break;
         }
         tc_fence_after();
+        const uint32_t t_sg = t_s + s_col(g);
         uint32_t r0[32], r1[32];
-        tmem_ld32(t_s, r0);
-        tmem_ld32(t_s + 32, r1);
+        tmem_ld32(t_sg, r0);
+        tmem_ld32(t_sg + 32, r1);
         tmem_ld_wait(r0);
         reg_fence(r1);
         // Masked steps: the causal diagonal, or (general mode) query blocks at
@@ -638,7 +668,7 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         };
         p_block(r0, 0);
         p_block(r1, 32);
-        tmem_st32(t_s, pw);
+        tmem_st32(t_sg, pw);
         tmem_st_wait();
         tc_fence_before();
         mbar_arrive(p_full);
@@ -675,7 +705,7 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         // its sequence is written row by row.
         if (!PACKED || j * 128 + 128 <= Nk) {
           uint8_t* stage = smem + C::kStageOff + ((g - 1) % NS) * C::kStageBytes;
-          stage_acc_row<D>(tmem + lane_base + (h == 0 ? 256 : 384), stage + (h == 0 ? C::kTile : 0),
+          stage_acc_row<D>(tmem + lane_base + (h == 0 ? 256 : C::kDkCol), stage + (h == 0 ? C::kTile : 0),
                            t, h == 0 ? 1.0f : scale);
           fence_proxy_async_smem();
         } else {
@@ -686,7 +716,7 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
           if (h == 0)
             store_acc_row<D>(tmem + lane_base + 256, dv + row_off, 1.0f, valid);
           else
-            store_acc_row<D>(tmem + lane_base + 384, dk + row_off, scale, valid);
+            store_acc_row<D>(tmem + lane_base + C::kDkCol, dk + row_off, scale, valid);
         }
         tc_fence_before();
         named_barrier_sync(1, 256);
