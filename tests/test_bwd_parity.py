@@ -79,6 +79,20 @@ def test_bwd_large_logits():
     check(workloads.small("bwd_q4", 1, 2, 2, 700, 128, True, q_mult=4.0, seed=21))
 
 
+@pytest.mark.parametrize("causal", [False, True])
+def test_bwd_d64_many_items(causal):
+    """d = 64 with more work items than SMs (dK/dV: 2 x 16 x 9 = 288, items of
+    odd and even step counts in a row), so the dK/dV kernel's alternating S^T
+    buffers run across item boundaries; three whole heads against the oracle."""
+    w = workloads.small(f"bwd_d64_items_c{int(causal)}", 2, 16, 16, 1100, 64, causal,
+                        seed=51 + int(causal))
+    q, k, v, do = workloads.make_inputs(w)
+    got = gpu_fwd_bwd(q, k, v, do, w.scale, w.causal)
+    picks = [(0, 0), (0, 9), (1, 15)]
+    refs = oracle.attention_backward(q, k, v, do, w.scale, w.causal, heads=picks)
+    assert_grads_close(got, refs, w.name, heads={"dq": picks, "dk": picks, "dv": picks})
+
+
 def test_bwd_c5_full_size_sampled_heads():
     """The training-step workload at full size; three whole heads compared exactly."""
     w = workloads.C5

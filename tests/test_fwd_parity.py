@@ -153,6 +153,27 @@ def test_causal_plan_shapes(w):
     assert torch.equal(o, o2) and torch.equal(lse, lse2)
 
 
+# d = 64 problems large enough for two-tile blocks (256 rows per CTA step),
+# dealt by the snake: unmasked and causal, with GQA.
+TWO_TILE_D64 = [workloads.small("d64_two_tile_B2_H16_N1200_nc", 2, 16, 16, 1200, 64, False, seed=41,
+                                backward=False),
+                workloads.small("d64_two_tile_B2_H16_KV8_N1500_c", 2, 16, 8, 1500, 64, True, seed=43,
+                                backward=False)]
+
+
+@pytest.mark.parametrize("w", TWO_TILE_D64, ids=lambda w: w.name)
+def test_d64_two_tile_blocks(w):
+    q, k, v = workloads.make_inputs(w, with_grad_out=False)
+    o, lse = gpu_fwd(q, k, v, w.scale, w.causal)
+    o_cpu, lse_cpu = o.float().cpu().numpy(), lse.cpu().numpy()
+    assert np.all(np.isfinite(o_cpu)) and np.all(np.isfinite(lse_cpu))
+    G = w.Hq // w.Hkv
+    for b, h in ((0, 0), (0, w.Hq - 1), (w.B - 1, w.Hq // 2)):
+        o_ref, lse_ref = oracle.attention_head(oracle.to_f64(q[b, h]), oracle.to_f64(k[b, h // G]),
+                                               oracle.to_f64(v[b, h // G]), w.scale, w.causal)
+        assert_fwd_close(o_cpu[b, h], lse_cpu[b, h], o_ref, lse_ref, f"{w.name} head ({b},{h})")
+
+
 def test_repeat_runs_are_bitwise_identical():
     w = workloads.small("det", 2, 4, 2, 700, 128, True, seed=3, backward=False)
     q, k, v = workloads.make_inputs(w, with_grad_out=False)
