@@ -160,6 +160,38 @@ def test_causal_plans_from_several_host_threads():
         assert torch.equal(o, refs[i][0]) and torch.equal(lse, refs[i][1]), (w, PLAN_SHAPES[i])
 
 
+def test_dependent_calls_back_to_back():
+    """Each forward reads the previous one's output (and a torch kernel sits
+    between some of them), with no synchronisation in between: the kernels are
+    launched with programmatic stream serialization and may start early, so
+    this checks that each one waits for its predecessor's results. Compared
+    bit for bit with the same chain synchronised after every call."""
+    q, k, v, do = _problem(21, N=900)
+    scale = 1.0 / 128 ** 0.5
+
+    def chain(sync):
+        x = q
+        outs = []
+        for i in range(6):
+            o, lse = ea.attn_fwd(x, k, v, causal=True, scale=scale)
+            if sync:
+                torch.cuda.synchronize()
+            outs.append((o, lse))
+            x = (o * 2.0) if i % 2 else o      # every other link through a torch kernel
+        dq, dk, dv = ea.attn_bwd(x, k, v, *ea.attn_fwd(x, k, v, causal=True, scale=scale), do,
+                                 causal=True, scale=scale)
+        outs.append((dq, dk, dv))
+        return outs
+
+    ref = chain(True)
+    got = chain(False)
+    torch.cuda.synchronize()
+    ea.attn_check_status()
+    for a, b in zip(got, ref):
+        for x, y in zip(a, b):
+            assert torch.equal(x, y)
+
+
 def test_calls_from_several_host_threads():
     problems = [_problem(10 + i, N=300 + 200 * i) for i in range(4)]
     refs = [_eager(*p) for p in problems]
